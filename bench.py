@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the LoSA hot path on B200.
+
+One step = one pass of the whole hot path over one layer of synthetic input:
+the construction step (dense attention + exact block masses, one kernel),
+the selection (frozen CSR pattern), then the workload's sparse steps on
+freshly drifted Q/K/V (10 for the Wan2.1-1.3B-shaped layer). The timed
+region holds K such steps with every input already resident in HBM; the
+inputs of one step (3.3 GB at the default workload) exceed the 126 MB L2.
+
+value = algorithmic TFLOP/s of the step:
+  construction pass 6*B*H*L_pad^2*d  (Q K^T twice and P V once),
+  each sparse step  4*b^2*d*nnz      (retained blocks only),
+divided by the step's device time. The JSON line also carries each part's
+own ms, TFLOP/s and fraction of the bf16 tensor-core peak, the selection and
+mass+select times, the sparse-vs-dense speedup and the kept fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl losa|reference]
+                    [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = ("block-sparse attn ms & TFLOP/s (retained blocks), % BF16 TC peak; "
+          "mass+select ms")
+DEFAULT_WORKLOAD = "wan2.1-1.3b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Kernels the library launches per call: dense_mass 1 (bf16 inputs), select 8, sparse 1.
+LAUNCHES_DENSE, LAUNCHES_SELECT, LAUNCHES_SPARSE = 1, 8, 1
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["losa", "reference"], default="losa")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--tau", type=float, default=0.99)
+    ap.add_argument("--sparse-steps", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="only run dense_mass x2, select, sparse_attn x2 (profiling)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_flops(wl, nnz, n_sparse):
+    """Algorithmic FLOPs of one step: construction pass + sparse steps."""
+    B, H, Lp, d, b = wl.batch, wl.heads, wl.seq_pad, wl.head_dim, wl.block
+    f_dense = 6.0 * B * H * Lp * Lp * d
+    f_sparse = 4.0 * b * b * d * nnz
+    return f_dense, f_sparse, f_dense + n_sparse * f_sparse
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                f = [x.strip() for x in r]
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+                for name, val in zip(names, f[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+
+def oracle_sample(wl, tau, n_sparse, budget_s, seed=4321):
+    """Times the oracle on a bounded sample of the workload: whole query
+    blocks of head 0 (dense rows, mass row, selection, and the sparse steps
+    of that block), until `budget_s` of CPU time. Returns (flops, seconds,
+    blocks, threads)."""
+    import numpy as np
+    import oracle as O
+    wl1 = dataclasses.replace(wl, heads=1, batch=1)
+    q, k, v = W.generate(wl1, dtype=torch.float32)
+    drifts = [W.drift(wl1, (q, k, v), step=s + 1, dtype=torch.float32) for s in range(n_sparse)]
+    L, Lp, b, d = wl.seq_len, wl.seq_pad, wl.block, wl.head_dim
+    scale = 1.0 / math.sqrt(d)
+    qh, kh, vh = (t[0, 0].double().numpy() for t in (q, k, v))
+    q4, k4 = qh[None, None], kh[None, None]
+    dh = [tuple(t[0, 0].double().numpy() for t in s) for s in drifts]
+    g = np.random.default_rng(seed)
+    order = g.permutation(wl.n_blocks)
+    flops, blocks = 0.0, 0
+    t0 = time.perf_counter()
+    for I in order:
+        rows = np.arange(I * b, min((I + 1) * b, L))
+        O.attention_rows(qh[rows], kh[:L], vh[:L], scale)
+        m = O.block_mass_row(q4, k4, L, b, scale, 0, 0, int(I))
+        kept, _, _ = O.select_row(O.to_fixed(m.astype(np.float32)).tolist(), tau)
+        keys = O.retained_keys(kept, b, L)
+        for (q2, k2, v2) in dh:
+            O.attention_rows(q2[rows], k2[keys], v2[keys], scale)
+        flops += 6.0 * b * Lp * d + n_sparse * 4.0 * b * b * d * len(kept)
+        blocks += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    secs = time.perf_counter() - t0
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=threads)
+    except Exception:
+        pass
+    return flops, secs, blocks, threads
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ reference arm
+
+def reference_arm(args, world, rank):
+    """The oracle as the reference implementation, on the host cores."""
+    if rank != 0:
+        return 0
+    wl = W.WORKLOADS[args.workload]
+    n_sparse = args.sparse_steps if args.sparse_steps is not None else max(1, wl.sparse_steps)
+    per_step = max(1.0, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, args.tau, n_sparse, per_step / 4)
+    tot_f, tot_s, tot_b, threads = 0.0, 0.0, 0, os.cpu_count()
+    for s in range(args.steps):
+        f, secs, blocks, threads = oracle_sample(wl, args.tau, n_sparse, per_step, seed=100 + s)
+        tot_f += f
+        tot_s += secs
+        tot_b += blocks
+    value = tot_f / tot_s / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "heads": wl.heads, "head_dim": wl.head_dim,
+                   "seq_len": wl.seq_len, "seq_pad": wl.seq_pad, "block": wl.block,
+                   "tau": args.tau, "sparse_steps": n_sparse},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{tot_b} whole query blocks of head 0 (dense rows, mass "
+                                   f"row, selection, {n_sparse} sparse steps), {per_step:.0f} s "
+                                   f"per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ LoSA arm
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = reference_arm(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+    import block_sparse_attention_losa_b200 as losa
+
+    wl = W.WORKLOADS[args.workload]
+    n_sparse = args.sparse_steps if args.sparse_steps is not None else max(1, wl.sparse_steps)
+    if args.ncu_case:
+        n_sparse = 1  # keeps the device footprint of a profiled run small
+    L, Lp, b, d, tau = wl.seq_len, wl.seq_pad, wl.block, wl.head_dim, args.tau
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # Inputs: construction Q/K/V plus n_sparse drifted sets, all resident.
+    qkv0 = W.generate(wl, device=dev)
+    sets, prev = [], qkv0
+    for s in range(n_sparse):
+        prev = W.drift(wl, prev, step=s + 1, device=dev)
+        sets.append(prev)
+    B, H = wl.batch, wl.heads
+    o_dense = torch.empty(B, H, Lp, d, device=dev, dtype=torch.bfloat16)
+    lse = torch.empty(B, H, Lp, device=dev, dtype=torch.float32)
+    mass = torch.empty(B, H, Lp // b, Lp // b, device=dev, dtype=torch.float32)
+    o_sparse = torch.empty(B, H, Lp, d, device=dev, dtype=torch.bfloat16)
+    lse_sparse = torch.empty(B, H, Lp, device=dev, dtype=torch.float32)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    if args.ncu_case:
+        for _ in range(2):
+            losa.dense_mass(*qkv0, L, b, out_dtype=torch.bfloat16, o=o_dense, lse=lse, mass=mass)
+        pat = losa.select(mass, b, tau)
+        for _ in range(2):
+            losa.sparse_attn(*sets[0], L, pat, out_dtype=torch.bfloat16, o=o_sparse,
+                             lse=lse_sparse)
+        torch.cuda.synchronize()
+        losa.check_status()
+        pat.close()
+        print("ncu case done", flush=True)
+        return 0
+
+    def one_step(record=None):
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(stream)
+        losa.dense_mass(*qkv0, L, b, out_dtype=torch.bfloat16, o=o_dense, lse=lse, mass=mass)
+        e1.record(stream)
+        pat = losa.select(mass, b, tau)
+        e2.record(stream)
+        sp = []
+        for (q2, k2, v2) in sets:
+            a, z = ev(), ev()
+            a.record(stream)
+            losa.sparse_attn(q2, k2, v2, L, pat, out_dtype=torch.bfloat16, o=o_sparse,
+                             lse=lse_sparse)
+            z.record(stream)
+            sp.append((a, z))
+        nnz, tiles_e = pat.nnz, pat.tile_entries
+        density = pat.density()
+        pat.close()
+        if record is not None:
+            record.append((e0, e1, e2, sp, nnz, tiles_e, density))
+
+    for _ in range(max(3, args.warmup)):
+        one_step()
+    torch.cuda.synchronize()
+    losa.check_status()
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    recs = []
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        one_step(recs)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    losa.check_status()
+
+    step_ms_local = t_start.elapsed_time(t_end) / args.steps
+    step_ms = max_over_ranks(step_ms_local, world)
+    dense_ms = statistics.mean(r[0].elapsed_time(r[1]) for r in recs)
+    select_ms = statistics.mean(r[1].elapsed_time(r[2]) for r in recs)
+    sparse_ms = statistics.mean(a.elapsed_time(z) for r in recs for (a, z) in r[3])
+    nnz, tile_entries, density = recs[-1][4], recs[-1][5], recs[-1][6]
+    f_dense, f_sparse, f_step = step_flops(wl, nnz, n_sparse)
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"]
+    value = world * f_step / (step_ms * 1e-3) / 1e12
+    sparse_tf = f_sparse / (sparse_ms * 1e-3) / 1e12
+    dense_tf = f_dense / (dense_ms * 1e-3) / 1e12
+    n_rows = B * H * (Lp // b)
+    # Dense attention time at the same shape (for the sparse-vs-dense ratio):
+    # the pass-1 share of the construction kernel, 4/6 of its work.
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "heads": H, "head_dim": d,
+                   "seq_len": L, "seq_pad": Lp, "block": b, "tau": tau,
+                   "sparse_steps": n_sparse, "l2": "inputs larger than L2 (3 x "
+                   f"{B * H * Lp * d * 2 / 1e6:.0f} MB per call)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "sparse_attn": {"ms": sparse_ms, "tflops": sparse_tf, "frac_of_peak": sparse_tf / peak,
+                        "retained_blocks": nnz, "kept_fraction": density,
+                        "tile_entries": tile_entries,
+                        "tile_overhead": tile_entries * (128 // b) / max(1, nnz)},
+        "dense_mass": {"ms": dense_ms, "tflops": dense_tf, "frac_of_peak": dense_tf / peak,
+                       "attn_equiv_tflops": 4.0 * B * H * L * L * d / (dense_ms * 1e-3) / 1e12},
+        "select_ms": select_ms, "mass_select_ms": dense_ms + select_ms,
+        "select_gbs": (4.0 * n_rows * (Lp // b) + 4.0 * nnz + 4.0 * (n_rows + 1)) /
+                      (select_ms * 1e-3) / 1e9,
+        "sparse_vs_dense_speedup": (dense_ms * 4.0 / 6.0) / sparse_ms,
+        "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": sparse_tf,
+                     "peak": peak, "unit": "TFLOP/s", "frac": sparse_tf / peak,
+                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": args.steps * (LAUNCHES_DENSE + LAUNCHES_SELECT + n_sparse * LAUNCHES_SPARSE),
+        "clocks": clock_info,
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_measure(losa, wl, qkv0, sets, args, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, secs, blocks, threads = oracle_sample(wl, tau, n_sparse, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": f / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{blocks} whole query blocks of head 0 (dense rows, mass row, "
+                      f"selection, {n_sparse} sparse steps) in {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_measure(losa, wl, qkv0, sets, args, world):
+    """The same step through the public API from pinned HOST buffers: each
+    step copies its inputs host->device and its outputs device->host inside
+    the timed region."""
+    L, Lp, b, d, tau = wl.seq_len, wl.seq_pad, wl.block, wl.head_dim, args.tau
+    stream = torch.cuda.current_stream()
+    host_sets = [tuple(t.cpu().pin_memory() for t in s) for s in [qkv0] + sets]
+    out_host = [torch.empty(wl.batch, wl.heads, Lp, d, dtype=torch.bfloat16).pin_memory()
+                for _ in host_sets]
+    h2d = sum(t.numel() * t.element_size() for s in host_sets for t in s)
+    d2h = sum(t.numel() * t.element_size() for t in out_host)
+
+    def step():
+        qd = [t.to("cuda", non_blocking=True) for t in host_sets[0]]
+        o, _, mass = losa.dense_mass(*qd, L, b, out_dtype=torch.bfloat16)
+        out_host[0].copy_(o, non_blocking=True)
+        pat = losa.select(mass, b, tau)
+        nnz = pat.nnz
+        for i, hs in enumerate(host_sets[1:], start=1):
+            sd = [t.to("cuda", non_blocking=True) for t in hs]
+            o2, _ = losa.sparse_attn(*sd, L, pat, out_dtype=torch.bfloat16, want_lse=False)
+            out_host[i].copy_(o2, non_blocking=True)
+        pat.close()
+        return nnz
+
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        nnz = step()
+    z.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(z) / args.e2e_steps, world)
+    _, _, f_step = step_flops(wl, nnz, len(host_sets) - 1)
+    return {"value": world * f_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

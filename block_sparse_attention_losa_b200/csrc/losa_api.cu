@@ -1,0 +1,268 @@
+// losa_api.cu - the library's C ABI: argument checks, the per-device status
+// word, the fp32 entry conversion, and pattern ownership.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "losa_device.cuh"
+#include "losa_internal.h"
+
+namespace losa {
+
+// One status word per device; kernels raise it on a timed-out wait or a
+// bad mass value, losa_check_status / losa_select read and clear it.
+__device__ int g_status_word;
+
+int* device_status_word() {
+  constexpr int kMaxDevices = 64;
+  static int* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+cudaMemPool_t device_pool() {
+  constexpr int kMaxDevices = 64;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
+void* pool_alloc(size_t bytes, cudaStream_t stream) {
+  cudaMemPool_t pool = device_pool();
+  if (!pool) return nullptr;
+  void* p = nullptr;
+  if (cudaMallocFromPoolAsync(&p, bytes ? bytes : 16, pool, stream) != cudaSuccess) return nullptr;
+  return p;
+}
+
+namespace {
+
+bool is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return false;
+  return major == 10 && minor == 0;
+}
+
+bool valid_dtype(int dt) { return dt == LOSA_BF16 || dt == LOSA_FP32; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by the attention calls.
+bool valid_attn_shape(int B, int H, int L, int L_pad, int d, int block) {
+  if (B < 1 || H < 1 || L < 1 || L > L_pad) return false;
+  if (d != 64 && d != 128) return false;
+  if (block != 32 && block != 64 && block != 128) return false;
+  if (L_pad % block != 0 || L_pad - L >= block) return false;
+  if (L_pad / block > 2047) return false;
+  if (int64_t(B) * H > 65535) return false;
+  return true;
+}
+
+// bf16 views of fp32 inputs, converted on the stream into temporaries.
+struct Bf16Inputs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* tmp = nullptr;
+  cudaStream_t s;
+  ~Bf16Inputs() {
+    if (tmp) cudaFreeAsync(tmp, s);
+  }
+};
+
+int prepare_inputs(Bf16Inputs& in, const void* q, const void* k, const void* v, int in_dtype,
+                   int64_t n_elem) {
+  if (in_dtype == LOSA_BF16) {
+    in.q = q;
+    in.k = k;
+    in.v = v;
+    return LOSA_OK;
+  }
+  const size_t bytes = size_t(n_elem) * 2;
+  in.tmp = pool_alloc(3 * bytes, in.s);
+  if (!in.tmp) return LOSA_ERR_NOMEM;
+  char* base = static_cast<char*>(in.tmp);
+  if (launch_f32_to_bf16(static_cast<const float*>(q), base, n_elem, in.s) != cudaSuccess ||
+      launch_f32_to_bf16(static_cast<const float*>(k), base + bytes, n_elem, in.s) != cudaSuccess ||
+      launch_f32_to_bf16(static_cast<const float*>(v), base + 2 * bytes, n_elem, in.s) != cudaSuccess)
+    return LOSA_ERR_CUDA;
+  in.q = base;
+  in.k = base + bytes;
+  in.v = base + 2 * bytes;
+  return LOSA_OK;
+}
+
+}  // namespace
+}  // namespace losa
+
+using namespace losa;
+
+extern "C" {
+
+int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype, int B, int H,
+                    int L, int L_pad, int d, int block, float scale, void* o, int out_dtype,
+                    float* lse, float* mass, void* stream) {
+  if (!q || !k || !v || !o || !lse || !mass) return LOSA_ERR_ARG;
+  if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LOSA_ERR_ARG;
+  if (!valid_attn_shape(B, H, L, L_pad, d, block)) return LOSA_ERR_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return LOSA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_ARG;
+  if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Bf16Inputs in;
+  in.s = s;
+  const int64_t n_elem = int64_t(B) * H * L_pad * d;
+  int st = prepare_inputs(in, q, k, v, in_dtype, n_elem);
+  if (st != LOSA_OK) return st;
+  if (launch_dense(in.q, in.k, in.v, B * H, L, L_pad, d, block, scale, o,
+                   out_dtype == LOSA_BF16, lse, mass, s) != cudaSuccess)
+    return LOSA_ERR_CUDA;
+  return LOSA_OK;
+}
+
+int losa_select(const float* mass, int B, int H, int n_blocks, int block, double tau,
+                losa_pattern** out, void* stream) {
+  if (out) *out = nullptr;
+  if (!mass || !out) return LOSA_ERR_ARG;
+  if (B < 1 || H < 1 || n_blocks < 1 || n_blocks > 2047) return LOSA_ERR_ARG;
+  if (block != 32 && block != 64 && block != 128) return LOSA_ERR_ARG;
+  if (int64_t(B) * H > 65535) return LOSA_ERR_ARG;
+  if (!(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_ARG;
+  if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
+  return build_pattern(mass, B, H, n_blocks, block, tau, out, static_cast<cudaStream_t>(stream));
+}
+
+int losa_pattern_info(const losa_pattern* p, losa_pattern_view* view) {
+  if (!p || !view) return LOSA_ERR_ARG;
+  view->B = p->B;
+  view->H = p->H;
+  view->n_blocks = p->n_blocks;
+  view->block = p->block;
+  view->nnz = p->nnz;
+  view->row_ptr = p->row_ptr;
+  view->col_idx = p->col_idx;
+  view->retained_fx = p->retained_fx;
+  view->total_fx = p->total_fx;
+  view->n_tiles = p->n_tiles;
+  view->tile_entries = p->tile_entries;
+  view->tile_ptr = p->tile_ptr;
+  view->tile_entry = p->tile_entry;
+  view->tile_order = p->tile_order;
+  return LOSA_OK;
+}
+
+int losa_pattern_export(const losa_pattern* p, int32_t* row_ptr, int32_t* col_idx,
+                        int64_t* retained_fx, int64_t* total_fx, int32_t* tile_ptr,
+                        int32_t* tile_entry, int32_t* tile_order, void* stream) {
+  if (!p) return LOSA_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t R = int64_t(p->B) * p->H * p->n_blocks;
+  struct Item {
+    void* dst;
+    const void* src;
+    size_t bytes;
+  } items[] = {{row_ptr, p->row_ptr, size_t(R + 1) * 4},
+               {col_idx, p->col_idx, size_t(p->nnz) * 4},
+               {retained_fx, p->retained_fx, size_t(R) * 8},
+               {total_fx, p->total_fx, size_t(R) * 8},
+               {tile_ptr, p->tile_ptr, size_t(p->n_tiles + 1) * 4},
+               {tile_entry, p->tile_entry, size_t(p->tile_entries) * 4},
+               {tile_order, p->tile_order, size_t(p->n_tiles) * 4}};
+  for (const Item& it : items) {
+    if (!it.dst || it.bytes == 0) continue;
+    if (cudaMemcpyAsync(it.dst, it.src, it.bytes, cudaMemcpyDefault, s) != cudaSuccess)
+      return LOSA_ERR_CUDA;
+  }
+  return cudaStreamSynchronize(s) == cudaSuccess ? LOSA_OK : LOSA_ERR_CUDA;
+}
+
+int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, int d, int L,
+                     float scale, const losa_pattern* p, void* o, int out_dtype, float* lse,
+                     void* stream) {
+  if (!q || !k || !v || !o || !p) return LOSA_ERR_ARG;
+  if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LOSA_ERR_ARG;
+  const int L_pad = p->n_blocks * p->block;
+  if (!valid_attn_shape(p->B, p->H, L, L_pad, d, p->block)) return LOSA_ERR_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return LOSA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_ARG;
+  if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Bf16Inputs in;
+  in.s = s;
+  const int64_t n_elem = int64_t(p->B) * p->H * L_pad * d;
+  int st = prepare_inputs(in, q, k, v, in_dtype, n_elem);
+  if (st != LOSA_OK) return st;
+  if (launch_sparse(in.q, in.k, in.v, d, L, scale, p, o, out_dtype == LOSA_BF16, lse, s) !=
+      cudaSuccess)
+    return LOSA_ERR_CUDA;
+  return LOSA_OK;
+}
+
+void losa_free(losa_pattern* p) {
+  if (!p) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->device);
+  if (p->fixed_mem) cudaFreeAsync(p->fixed_mem, p->stream);
+  if (p->list_mem) cudaFreeAsync(p->list_mem, p->stream);
+  cudaSetDevice(prev);
+  delete p;
+}
+
+int losa_check_status(void* stream) {
+  int* w = device_status_word();
+  if (!w) return LOSA_ERR_CUDA;
+  int h = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, w, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return LOSA_ERR_CUDA;
+  if (h != kStatusOk) {
+    const int zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return LOSA_ERR_CUDA;
+    return h == kStatusBadMass ? LOSA_ERR_MASS : LOSA_ERR_TIMEOUT;
+  }
+  return LOSA_OK;
+}
+
+const char* losa_strerror(int status) {
+  switch (status) {
+    case LOSA_OK: return "ok";
+    case LOSA_ERR_ARG: return "invalid argument";
+    case LOSA_ERR_CUDA: return "CUDA runtime error";
+    case LOSA_ERR_NOMEM: return "device allocation failed";
+    case LOSA_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case LOSA_ERR_MASS: return "mass entry is NaN, Inf, negative or >= 2";
+    case LOSA_ERR_UNSUPPORTED: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+const char* losa_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+// losa_attention.cu - host launchers of the attention kernels: TMA tensor
+// maps, kernel instantiation per (head dim, key tile, output dtype), and the
+// fp32 -> bf16 entry conversion.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "losa_attention.cuh"
+#include "losa_internal.h"
+
+namespace losa {
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q{};
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [BH, L_pad, d] bf16 viewed as a 3D tensor (d innermost), loaded in
+// 64-column (128 B) slabs of `box_rows` rows with the 128-byte swizzle the
+// MMA descriptors expect. Rows past L_pad read as zero.
+bool make_map(CUtensorMap* map, const void* base, int BH, int L_pad, int d, int box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(L_pad), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(L_pad) * d * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BN, int NS, bool kDense, bool kOutBf16>
+cudaError_t run(const void* q, const void* k, const void* v, int BH, const AttnParams& p,
+                dim3 grid, cudaStream_t stream) {
+  using Lay = AttnLayout<D, BN, NS>;
+  auto kern = attn_kernel<D, BN, NS, kDense, kOutBf16>;
+  // Cheap, and per device: set on every launch.
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM_ALLOC);
+  if (err != cudaSuccess) return err;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, BH, p.L_pad, D, 128) || !make_map(&tk, k, BH, p.L_pad, D, BN) ||
+      !make_map(&tv, v, BH, p.L_pad, D, BN))
+    return cudaErrorInvalidValue;
+  kern<<<grid, 192, Lay::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+__global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
+                                   int64_t n4) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float4 x = src[i];
+    uint2 y;
+    y.x = pack_bf16x2(x.x, x.y);
+    y.y = pack_bf16x2(x.z, x.w);
+    dst[i] = y;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {
+  // n is a multiple of 64 (d in {64, 128}); 16-byte aligned pointers.
+  const int64_t n4 = n / 4;
+  const int grid = int(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
+  f32_to_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(src),
+                                               reinterpret_cast<uint2*>(dst), n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, int L, int L_pad,
+                         int d, int block, float scale, void* o, bool out_bf16, float* lse,
+                         float* mass, cudaStream_t stream) {
+  AttnParams p{};
+  p.L = L;
+  p.L_pad = L_pad;
+  p.n_qt = (L_pad + 127) / 128;
+  p.n_kv = (L_pad + 127) / 128;
+  p.block = block;
+  p.n_blocks = L_pad / block;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = o;
+  p.lse = lse;
+  p.mass = mass;
+  p.status = device_status_word();
+  if (!p.status) return cudaErrorInvalidDevice;
+  const dim3 grid(p.n_qt, BH);
+  if (d == 128) {
+    return out_bf16 ? run<128, 128, 2, true, true>(q, k, v, BH, p, grid, stream)
+                    : run<128, 128, 2, true, false>(q, k, v, BH, p, grid, stream);
+  }
+  return out_bf16 ? run<64, 128, 3, true, true>(q, k, v, BH, p, grid, stream)
+                  : run<64, 128, 3, true, false>(q, k, v, BH, p, grid, stream);
+}
+
+cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, int L,
+                          float scale, const losa_pattern* pat, void* o, bool out_bf16,
+                          float* lse, cudaStream_t stream) {
+  AttnParams p{};
+  p.L = L;
+  p.L_pad = pat->n_blocks * pat->block;
+  p.n_qt = pat->n_qt;
+  p.n_kv = 0;
+  p.block = pat->block;
+  p.n_blocks = pat->n_blocks;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = o;
+  p.lse = lse;
+  p.mass = nullptr;
+  p.tile_ptr = pat->tile_ptr;
+  p.tile_entry = pat->tile_entry;
+  p.tile_order = pat->tile_order;
+  p.status = device_status_word();
+  if (!p.status) return cudaErrorInvalidDevice;
+  const int BH = pat->B * pat->H;
+  const dim3 grid(unsigned(pat->n_tiles));
+  if (pat->n_tiles == 0) return cudaSuccess;
+#define LOSA_SPARSE_CASE(D_, BN_, NS_)                                                    \
+  if (d == D_ && pat->block == BN_)                                                      \
+    return out_bf16 ? run<D_, BN_, NS_, false, true>(q, k, v, BH, p, grid, stream)      \
+                    : run<D_, BN_, NS_, false, false>(q, k, v, BH, p, grid, stream);
+  LOSA_SPARSE_CASE(128, 128, 2)
+  LOSA_SPARSE_CASE(128, 64, 4)
+  LOSA_SPARSE_CASE(128, 32, 4)
+  LOSA_SPARSE_CASE(64, 128, 3)
+  LOSA_SPARSE_CASE(64, 64, 4)
+  LOSA_SPARSE_CASE(64, 32, 4)
+#undef LOSA_SPARSE_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace losa

@@ -1,0 +1,61 @@
+// losa_internal.h - host-side declarations shared by the library's
+// translation units (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/losa.h"
+
+struct losa_pattern {
+  int B, H, n_blocks, block;
+  int device;
+  cudaStream_t stream;   // the stream the pattern was built on (frees go there)
+  void* fixed_mem;       // row_ptr, tile_ptr, tile_order, retained_fx, total_fx
+  void* list_mem;        // col_idx, tile_entry
+  int64_t nnz;
+  int64_t n_tiles;       // B*H*n_qt
+  int64_t tile_entries;  // total union entries
+  int n_qt;              // 128-row query tiles per head
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int64_t* retained_fx;
+  int64_t* total_fx;
+  int32_t* tile_ptr;
+  int32_t* tile_entry;
+  int32_t* tile_order;
+};
+
+namespace losa {
+
+// Device status word of the current device (lazily resolved per device).
+int* device_status_word();
+
+// The library's stream-ordered memory pool on the current device (created
+// on first use, release threshold at maximum so steady-state calls reuse
+// memory instead of mapping it again). Returns nullptr on failure.
+cudaMemPool_t device_pool();
+
+// Stream-ordered allocation from device_pool(); nullptr on failure.
+void* pool_alloc(size_t bytes, cudaStream_t stream);
+
+// Runs the dense two-pass construction kernel. q/k/v are bf16 device
+// pointers; the arguments were validated by the caller.
+cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, int L, int L_pad,
+                         int d, int block, float scale, void* o, bool out_bf16, float* lse,
+                         float* mass, cudaStream_t stream);
+
+// Runs the block-sparse kernel over pattern p (validated by the caller).
+cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, int L,
+                          float scale, const losa_pattern* p, void* o, bool out_bf16,
+                          float* lse, cudaStream_t stream);
+
+// fp32 -> bf16 (round to nearest even) of n elements.
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
+
+// Builds the frozen pattern from a mass map (validated by the caller).
+// Returns a losa_status.
+int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
+                  losa_pattern** out, cudaStream_t stream);
+
+}  // namespace losa

@@ -1,0 +1,400 @@
+// losa_select.cu - the selection step of LoSA on the GPU: per (b, h, query
+// block), the smallest key-block set whose cumulative mass reaches tau
+// (ubos.tech LoSA post, "How It Works in Practice", Phase 2 - Block Mask
+// Generation: sort key blocks by descending mass and accumulate until the
+// threshold is met; LoSA abstract, arXiv 2608.12032: "keeps, for each head
+// and query block, the smallest key/value block set meeting the threshold").
+//
+// All of it is integer work on 64-bit fixed-point masses x = round(m * 2^48),
+// so the result is bit-exact. Instead of sorting each row, the kernel finds
+// the cut with an MSD radix select over the sort keys
+//     key(J) = ((2^49 - 1 - x_J) << 11) | J          (< 2^60, unique per row)
+// whose ascending order is (x desc, J asc): it narrows 8 bits at a time to
+// the bucket where the running sum first reaches the threshold, keeping
+// per-bucket sums and counts in shared memory. The kept set is then
+// {J : key(J) <= cut key}, written out in ascending J.
+#include <cub/block/block_reduce.cuh>
+#include <cub/block/block_scan.cuh>
+
+#include <cstdio>
+#include <vector>
+
+#include "losa_device.cuh"
+#include "losa_internal.h"
+
+namespace losa {
+namespace {
+
+constexpr int kSelThreads = 256;
+constexpr int kMaxBlocks = 2047;                               // n <= 2047: J fits 11 bits
+constexpr int kKeysPerThread = (kMaxBlocks + kSelThreads) / kSelThreads;  // 8
+constexpr unsigned long long kXMax = (1ull << 49) - 1;          // masses in [0, 2)
+constexpr unsigned long long kNoKey = ~0ull;
+
+// x = round(m * 2^48) (ties to even; exact, as m * 2^48 only shifts the
+// exponent). Returns false for NaN, Inf, negative or >= 2.
+__device__ __forceinline__ bool to_fixed(float m, long long& x) {
+  if (!(m >= 0.f && m < 2.f)) {
+    x = 0;
+    return false;
+  }
+  x = __double2ll_rn(double(m) * 281474976710656.0);
+  return true;
+}
+
+__device__ __forceinline__ unsigned long long sort_key(long long x, int J) {
+  return ((kXMax - (unsigned long long)x) << 11) | (unsigned long long)J;
+}
+
+// 2^48 * C >= tau_fx * S, exactly.
+__device__ __forceinline__ bool reaches(unsigned long long C, unsigned long long tau_fx,
+                                        unsigned long long S) {
+  return ((unsigned __int128)C << 48) >= (unsigned __int128)tau_fx * S;
+}
+
+// One CTA per row: the cut key, kept count, kept and total fixed-point mass.
+__global__ void __launch_bounds__(kSelThreads)
+    select_cut_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
+                      unsigned long long* __restrict__ cut_key, int* __restrict__ count,
+                      long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
+                      int* status) {
+  using Reduce = cub::BlockReduce<unsigned long long, kSelThreads>;
+  __shared__ typename Reduce::TempStorage red_tmp;
+  __shared__ unsigned long long bsum[256];
+  __shared__ unsigned int bcnt[256];
+  __shared__ unsigned long long sh_S, sh_acc, sh_hi, sh_cut;
+  __shared__ int sh_done, sh_bad;
+
+  const int row = blockIdx.x;
+  const float* mrow = mass + size_t(row) * n;
+  unsigned long long key[kKeysPerThread];
+  long long xs[kKeysPerThread];
+  bool bad = false;
+  unsigned long long local = 0;
+#pragma unroll
+  for (int i = 0; i < kKeysPerThread; ++i) {
+    const int J = threadIdx.x + i * kSelThreads;
+    key[i] = kNoKey;
+    xs[i] = 0;
+    if (J < n) {
+      long long x;
+      bad |= !to_fixed(mrow[J], x);
+      xs[i] = x;
+      key[i] = sort_key(x, J);
+      local += (unsigned long long)x;
+    }
+  }
+  if (threadIdx.x == 0) sh_bad = 0;
+  __syncthreads();
+  if (bad) sh_bad = 1;
+  const unsigned long long S_part = Reduce(red_tmp).Sum(local);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    sh_S = S_part;
+    sh_acc = 0;
+    sh_hi = 0;
+    sh_done = 0;
+    if (sh_bad) atomicCAS(status, kStatusOk, kStatusBadMass);
+  }
+  __syncthreads();
+  const unsigned long long S = sh_S;
+
+  // MSD radix select, 8 bits per pass from bit 56 down.
+  int shift = 56;
+  for (; shift >= 0; shift -= 8) {
+    bsum[threadIdx.x] = 0;
+    bcnt[threadIdx.x] = 0;
+    __syncthreads();
+    const unsigned long long hi = sh_hi;
+#pragma unroll
+    for (int i = 0; i < kKeysPerThread; ++i) {
+      if (key[i] != kNoKey && (shift == 56 || (key[i] >> (shift + 8)) == hi)) {
+        const int d = int((key[i] >> shift) & 0xFF);
+        atomicAdd(&bsum[d], (unsigned long long)xs[i]);
+        atomicAdd(&bcnt[d], 1u);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // Warp 0: first non-empty bucket where the running sum reaches the
+      // threshold. Lane t owns buckets [8t, 8t + 8).
+      const int t = threadIdx.x;
+      unsigned long long my = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) my += bsum[t * 8 + j];
+      unsigned long long incl = my;  // inclusive warp scan
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (t >= off) incl += v;
+      }
+      const unsigned long long acc = sh_acc;
+      unsigned long long run = acc + incl - my;  // sum of buckets before mine
+      int found = 256;
+      unsigned long long before = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int d = t * 8 + j;
+        const unsigned long long after = run + bsum[d];
+        if (found == 256 && bcnt[d] > 0 && reaches(after, tau_fx, S)) {
+          found = d;
+          before = run;
+        }
+        run = after;
+      }
+      const int first = __reduce_min_sync(0xffffffffu, unsigned(found));
+      if (found == first && found < 256) {
+        sh_acc = before;
+        sh_hi = (sh_hi << 8) | unsigned(found);
+        sh_done = (bcnt[found] == 1) ? 1 : 0;
+      }
+    }
+    __syncthreads();
+    if (sh_done) break;
+  }
+  // The cut key: the single key left in the chosen bucket.
+  const int s_final = shift < 0 ? 0 : shift;
+  if (threadIdx.x == 0) sh_cut = kNoKey;
+  __syncthreads();
+  const unsigned long long hi = sh_hi;
+#pragma unroll
+  for (int i = 0; i < kKeysPerThread; ++i)
+    if (key[i] != kNoKey && (key[i] >> s_final) == hi) sh_cut = key[i];
+  __syncthreads();
+  const unsigned long long cut = sh_cut;
+  unsigned long long kept = 0, kept_n = 0;
+#pragma unroll
+  for (int i = 0; i < kKeysPerThread; ++i) {
+    if (key[i] <= cut) {
+      kept += (unsigned long long)xs[i];
+      kept_n += 1;
+    }
+  }
+  const unsigned long long C = Reduce(red_tmp).Sum(kept);
+  __syncthreads();
+  const unsigned long long K = Reduce(red_tmp).Sum(kept_n);
+  if (threadIdx.x == 0) {
+    cut_key[row] = cut;
+    count[row] = int(K);
+    retained_fx[row] = (long long)C;
+    total_fx[row] = (long long)S;
+  }
+}
+
+// Per 128-row tile (128/block query blocks): which key blocks each query
+// block keeps, as a bitmask m_J (bit q = q-th query block of the tile).
+__device__ __forceinline__ unsigned tile_mask(const float* __restrict__ mass,
+                                              const unsigned long long* __restrict__ cut_key,
+                                              int n, int row0, int nq, int J) {
+  unsigned m = 0;
+  for (int q = 0; q < nq; ++q) {
+    const int r = row0 + q;
+    long long x;
+    to_fixed(mass[size_t(r) * n + J], x);
+    if (sort_key(x, J) <= cut_key[r]) m |= 1u << q;
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    tile_count_kernel(const float* __restrict__ mass, const unsigned long long* __restrict__ cut_key,
+                      int n, int qpt, int n_qt, int* __restrict__ tile_count) {
+  using Reduce = cub::BlockReduce<int, kSelThreads>;
+  __shared__ typename Reduce::TempStorage tmp;
+  const int t = blockIdx.x;
+  const int bh = t / n_qt, qt = t % n_qt;
+  const int I0 = qt * qpt;
+  const int nq = min(qpt, n - I0);
+  const int row0 = bh * n + I0;
+  int c = 0;
+  for (int J = threadIdx.x; J < n; J += kSelThreads)
+    c += tile_mask(mass, cut_key, n, row0, nq, J) != 0;
+  const int total = Reduce(tmp).Sum(c);
+  if (threadIdx.x == 0) tile_count[t] = total;
+}
+
+// Writes each query block's kept key blocks (ascending) into col_idx and the
+// tile's union entries (J | mask << 16, ascending J) into tile_entry.
+// Counts of one 256-wide chunk are scanned together, packed in 10-bit fields:
+// fields 0..3 = query blocks of the tile, field 4 = the union.
+__global__ void __launch_bounds__(kSelThreads)
+    tile_write_kernel(const float* __restrict__ mass, const unsigned long long* __restrict__ cut_key,
+                      int n, int qpt, int n_qt, const int* __restrict__ row_ptr,
+                      const int* __restrict__ tile_ptr, int* __restrict__ col_idx,
+                      int* __restrict__ tile_entry) {
+  using Scan = cub::BlockScan<unsigned long long, kSelThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  const int t = blockIdx.x;
+  const int bh = t / n_qt, qt = t % n_qt;
+  const int I0 = qt * qpt;
+  const int nq = min(qpt, n - I0);
+  const int row0 = bh * n + I0;
+  int base[4];
+  for (int q = 0; q < 4; ++q) base[q] = (q < nq) ? row_ptr[row0 + q] : 0;
+  int ubase = tile_ptr[t];
+  for (int c0 = 0; c0 < n; c0 += kSelThreads) {
+    const int J = c0 + threadIdx.x;
+    const unsigned m = (J < n) ? tile_mask(mass, cut_key, n, row0, nq, J) : 0u;
+    unsigned long long v = 0;
+    for (int q = 0; q < 4; ++q) v |= (unsigned long long)((m >> q) & 1u) << (10 * q);
+    v |= (unsigned long long)(m != 0) << 40;
+    unsigned long long ex, tot;
+    Scan(tmp).ExclusiveSum(v, ex, tot);
+    __syncthreads();
+    for (int q = 0; q < nq; ++q)
+      if ((m >> q) & 1u) col_idx[base[q] + int((ex >> (10 * q)) & 1023)] = J;
+    if (m) tile_entry[ubase + int((ex >> 40) & 1023)] = J | int(m << 16);
+    for (int q = 0; q < 4; ++q) base[q] += int((tot >> (10 * q)) & 1023);
+    ubase += int((tot >> 40) & 1023);
+  }
+}
+
+// Exclusive scan of n ints into out[0..n] (out[n] = total), one CTA.
+__global__ void __launch_bounds__(1024) scan_kernel(const int* __restrict__ in, int n,
+                                                    int* __restrict__ out) {
+  using Scan = cub::BlockScan<int, 1024>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < n; c0 += 1024) {
+    const int i = c0 + threadIdx.x;
+    const int v = (i < n) ? in[i] : 0;
+    int ex, tot;
+    Scan(tmp).ExclusiveSum(v, ex, tot);
+    const int c = carry;
+    if (i < n) out[i] = c + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry = c + tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[n] = carry;
+}
+
+// Tiles ordered by entry count, largest first (longest-processing-time
+// order for the sparse kernel's block scheduler). Counting sort on
+// (n - count); order among equal counts is unspecified.
+__global__ void order_hist_kernel(const int* __restrict__ tile_count, int T, int n,
+                                  int* __restrict__ hist) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x)
+    atomicAdd(&hist[n - tile_count[t]], 1);
+}
+
+__global__ void order_scatter_kernel(const int* __restrict__ tile_count, int T, int n,
+                                     int* __restrict__ cursor, int* __restrict__ order) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x)
+    order[atomicAdd(&cursor[n - tile_count[t]], 1)] = t;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
+                  losa_pattern** out, cudaStream_t stream) {
+  const int BH = B * H;
+  const int64_t R = int64_t(BH) * n;
+  const int L_pad = n * block;
+  const int n_qt = (L_pad + 127) / 128;
+  const int qpt = 128 / block;
+  const int64_t T = int64_t(BH) * n_qt;
+  const unsigned long long tau_fx = (unsigned long long)llrint(tau * 281474976710656.0);
+  int* status = device_status_word();
+  if (!status) return LOSA_ERR_CUDA;
+
+  losa_pattern* p = new losa_pattern{};
+  p->B = B;
+  p->H = H;
+  p->n_blocks = n;
+  p->block = block;
+  p->n_qt = n_qt;
+  p->n_tiles = T;
+  p->stream = stream;
+  cudaGetDevice(&p->device);
+
+  // Pattern arrays of known size: one allocation.
+  const size_t o_row = 0;
+  const size_t o_tptr = o_row + align256((R + 1) * 4);
+  const size_t o_tord = o_tptr + align256((T + 1) * 4);
+  const size_t o_ret = o_tord + align256(T * 4);
+  const size_t o_tot = o_ret + align256(R * 8);
+  const size_t fixed_bytes = o_tot + align256(R * 8);
+  // Scratch: cut keys, row counts, tile counts, histogram, cursor.
+  const size_t s_cut = 0;
+  const size_t s_cnt = s_cut + align256(R * 8);
+  const size_t s_tcnt = s_cnt + align256(R * 4);
+  const size_t s_hist = s_tcnt + align256(T * 4);
+  const size_t s_cur = s_hist + align256((n + 1) * 4);
+  const size_t scratch_bytes = s_cur + align256((n + 2) * 4);
+
+  char* fixed = static_cast<char*>(pool_alloc(fixed_bytes, stream));
+  char* scratch = static_cast<char*>(pool_alloc(scratch_bytes, stream));
+  auto fail = [&](int code) {
+    if (fixed) cudaFreeAsync(fixed, stream);
+    if (scratch) cudaFreeAsync(scratch, stream);
+    if (p->list_mem) cudaFreeAsync(p->list_mem, stream);
+    delete p;
+    return code;
+  };
+  if (!fixed || !scratch) return fail(LOSA_ERR_NOMEM);
+  p->fixed_mem = fixed;
+  p->row_ptr = reinterpret_cast<int32_t*>(fixed + o_row);
+  p->tile_ptr = reinterpret_cast<int32_t*>(fixed + o_tptr);
+  p->tile_order = reinterpret_cast<int32_t*>(fixed + o_tord);
+  p->retained_fx = reinterpret_cast<int64_t*>(fixed + o_ret);
+  p->total_fx = reinterpret_cast<int64_t*>(fixed + o_tot);
+  auto* cut = reinterpret_cast<unsigned long long*>(scratch + s_cut);
+  auto* cnt = reinterpret_cast<int*>(scratch + s_cnt);
+  auto* tcnt = reinterpret_cast<int*>(scratch + s_tcnt);
+  auto* hist = reinterpret_cast<int*>(scratch + s_hist);
+  auto* cursor = reinterpret_cast<int*>(scratch + s_cur);
+
+  select_cut_kernel<<<unsigned(R), kSelThreads, 0, stream>>>(mass, n, tau_fx, cut, cnt,
+                                                              (long long*)p->retained_fx,
+                                                              (long long*)p->total_fx, status);
+  tile_count_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(mass, cut, n, qpt, n_qt, tcnt);
+  scan_kernel<<<1, 1024, 0, stream>>>(cnt, int(R), p->row_ptr);
+  scan_kernel<<<1, 1024, 0, stream>>>(tcnt, int(T), p->tile_ptr);
+  cudaMemsetAsync(hist, 0, (n + 1) * sizeof(int), stream);
+  const int og = int(std::min<int64_t>((T + 255) / 256, 1024));
+  order_hist_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n, hist);
+  scan_kernel<<<1, 1024, 0, stream>>>(hist, n + 1, cursor);
+  order_scatter_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n, cursor, p->tile_order);
+  if (cudaGetLastError() != cudaSuccess) return fail(LOSA_ERR_CUDA);
+
+  // The one host synchronisation: CSR sizes and the mass check.
+  int totals[2] = {0, 0};
+  int host_status = 0;
+  if (cudaMemcpyAsync(&totals[0], p->row_ptr + R, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(&totals[1], p->tile_ptr + T, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return fail(LOSA_ERR_CUDA);
+  if (host_status != kStatusOk) {
+    const int zero = 0;
+    cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(host_status == kStatusBadMass ? LOSA_ERR_MASS : LOSA_ERR_TIMEOUT);
+  }
+  p->nnz = totals[0];
+  p->tile_entries = totals[1];
+  const size_t list_bytes = align256(size_t(p->nnz) * 4) + align256(size_t(p->tile_entries) * 4);
+  char* lists = static_cast<char*>(pool_alloc(list_bytes, stream));
+  if (!lists) return fail(LOSA_ERR_NOMEM);
+  p->list_mem = lists;
+  p->col_idx = reinterpret_cast<int32_t*>(lists);
+  p->tile_entry = reinterpret_cast<int32_t*>(lists + align256(size_t(p->nnz) * 4));
+  tile_write_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(
+      mass, cut, n, qpt, n_qt, p->row_ptr, p->tile_ptr, p->col_idx, p->tile_entry);
+  if (cudaGetLastError() != cudaSuccess) {
+    p->fixed_mem = nullptr;
+    return fail(LOSA_ERR_CUDA);
+  }
+  cudaFreeAsync(scratch, stream);
+  *out = p;
+  return LOSA_OK;
+}
+
+}  // namespace losa

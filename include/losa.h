@@ -1,0 +1,202 @@
+/*
+ * losa.h - C ABI of the LoSA retained-mass block-sparse attention library
+ * (B200, sm_100a).
+ *
+ * The method (LoSA: Near-Lossless Sparse Attention for Training-Free Video
+ * Diffusion Acceleration, arXiv 2608.12032) runs in three phases, and each
+ * phase is one call here:
+ *
+ *   losa_dense_mass   one early dense attention step that also measures the
+ *                     exact attention mass of every (head, query block, key
+ *                     block) pair (ubos.tech LoSA post, "How It Works in
+ *                     Practice", Phase 1 - Dense Calibration; LoSA abstract:
+ *                     "measures exact block attention masses at one early
+ *                     dense step").
+ *   losa_select       per head and query block, the smallest key-block set
+ *                     whose cumulative mass reaches tau (Phase 2 - Block
+ *                     Mask Generation; legiblepapers.com LoSA page, "Summary
+ *                     & Methodology Analysis": default tau = 0.99), frozen
+ *                     into a CSR pattern the library owns.
+ *   losa_sparse_attn  every later step: attention of fresh Q/K/V over the
+ *                     frozen retained key blocks only (Phase 3 - Repeated
+ *                     Sparse Inference; legiblepapers.com: Q, K, V are
+ *                     recomputed, the indices are not).
+ *   losa_free         releases a pattern.
+ *
+ * Conventions shared by every call:
+ *   - Tensors are caller-owned DEVICE memory on the current CUDA device,
+ *     contiguous, row-major. Q, K, V, O are [B, H, L_pad, d]; lse is
+ *     [B, H, L_pad]; the mass map is [B, H, n, n] with n = L_pad / block.
+ *     Base pointers of Q, K, V must be 16-byte aligned.
+ *   - Token rows i >= L are padding: keys there take no weight, and query
+ *     rows there get O = 0 and lse = -inf and are left out of the masses.
+ *     L_pad must be a multiple of the block size, and L_pad - L < block.
+ *   - Attention is bidirectional: softmax(scale * q k^T) over the valid keys.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     stream-ordered and return without a host synchronisation, except
+ *     losa_select (one synchronisation, to size the CSR) and
+ *     losa_check_status.
+ *   - Every call returns LOSA_OK (0) or a negative losa_status; it checks
+ *     its arguments on the host before touching the device and then leaves
+ *     outputs untouched on LOSA_ERR_ARG.
+ *   - Supported: d in {64, 128}; block in {32, 64, 128}; n <= 2047;
+ *     B*H <= 65535; an sm_100 device.
+ *   - The library keeps no global state besides one device status word per
+ *     device (set by a kernel that ran out of a bounded wait, or by a bad
+ *     mass value) and its CUDA function handles. Calls on different streams
+ *     are independent.
+ */
+#ifndef LOSA_H_
+#define LOSA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LOSA_BF16 = 0, /* bfloat16 */
+  LOSA_FP32 = 1  /* float32; inputs are rounded to bf16 (nearest even) on entry */
+} losa_dtype;
+
+typedef enum {
+  LOSA_OK = 0,
+  LOSA_ERR_ARG = -1,         /* bad argument: shape, dtype, null pointer, tau */
+  LOSA_ERR_CUDA = -2,        /* a CUDA runtime call failed */
+  LOSA_ERR_NOMEM = -3,       /* device allocation failed */
+  LOSA_ERR_TIMEOUT = -4,     /* a kernel gave up a bounded wait (see losa_check_status) */
+  LOSA_ERR_MASS = -5,        /* a mass entry is NaN, Inf, negative or >= 2 */
+  LOSA_ERR_UNSUPPORTED = -6  /* the current device is not sm_100 */
+} losa_status;
+
+/* A frozen block pattern: opaque, owned by the library, freed by losa_free. */
+typedef struct losa_pattern losa_pattern;
+
+/* Read-only view of a pattern. All pointers are DEVICE pointers owned by the
+ * pattern and valid until losa_free. Rows are ordered (b, h, I) row-major,
+ * R = B*H*n rows. */
+typedef struct {
+  int B, H, n_blocks, block;
+  int64_t nnz;                 /* retained (query block, key block) pairs */
+  const int32_t* row_ptr;      /* [R + 1], row_ptr[0] = 0, row_ptr[R] = nnz */
+  const int32_t* col_idx;      /* [nnz], ascending key-block index within a row */
+  const int64_t* retained_fx;  /* [R], sum of the kept fixed-point masses */
+  const int64_t* total_fx;     /* [R], sum of all fixed-point masses of the row */
+  /* Work list of the sparse kernel: 128-query-row tiles (128/block query
+   * blocks each). A tile's entries are the union of its query blocks'
+   * retained key blocks, ascending; entry = J | (m << 16), bit q of m set
+   * when the tile's q-th query block keeps key block J. */
+  int64_t n_tiles;
+  int64_t tile_entries;
+  const int32_t* tile_ptr;     /* [n_tiles + 1] */
+  const int32_t* tile_entry;   /* [tile_entries] */
+  const int32_t* tile_order;   /* [n_tiles], tiles by entry count, largest first */
+} losa_pattern_view;
+
+/*
+ * losa_dense_mass - construction step: dense attention plus the exact block
+ * attention mass (Phase 1 - Dense Calibration, ubos.tech LoSA post; LoSA
+ * abstract).
+ *
+ *   q, k, v    [B, H, L_pad, d] device, dtype in_dtype.
+ *   o          [B, H, L_pad, d] device, dtype out_dtype:
+ *              O = softmax(scale * Q K^T over keys j < L) V.
+ *   lse        [B, H, L_pad] fp32 device: lse_i = log sum_{j<L} exp(scale q_i.k_j).
+ *   mass       [B, H, n, n] fp32 device, n = L_pad / block:
+ *              mass[b,h,I,J] = (1/|I|) sum_{i in I, i<L} sum_{j in J}
+ *                              exp(scale q_i.k_j - lse_i),
+ *              |I| = valid query rows of block I; each row sums to 1.
+ *   One kernel with two passes over the key tiles: a flash forward that
+ *   leaves O and lse, then a recompute of Q K^T that sums exp(s - lse) into
+ *   the block masses. o, lse and mass must not alias the inputs.
+ *   Returns LOSA_ERR_ARG for: a null pointer, B, H < 1, L < 1, L > L_pad,
+ *   L_pad % block != 0, L_pad - L >= block, d not in {64, 128}, block not in
+ *   {32, 64, 128}, n > 2047, B*H > 65535, a dtype out of range, scale not
+ *   finite and > 0.
+ */
+int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype,
+                    int B, int H, int L, int L_pad, int d, int block, float scale,
+                    void* o, int out_dtype, float* lse, float* mass, void* stream);
+
+/*
+ * losa_select - smallest key-block set per (b, h, query block) whose
+ * cumulative mass reaches tau (Phase 2 - Block Mask Generation; LoSA
+ * abstract; legiblepapers.com FAQ Q4).
+ *
+ *   mass      [B, H, n, n] fp32 device (as written by losa_dense_mass).
+ *   tau       in (0, 1]; the method's default is 0.99.
+ *   out       receives a new pattern on LOSA_OK, else NULL.
+ *
+ *   Per row: x_J = round(mass_J * 2^48) as int64 (ties to even); order the
+ *   key blocks by (x desc, J asc); C_k = prefix sums; S = sum x; keep the
+ *   first k >= 1 blocks with 2^48 * C_k >= round(tau * 2^48) * S, compared
+ *   exactly in 128-bit integers. The kept set is stored ascending. Integer
+ *   work throughout, so the result is bit-exact.
+ *   Allocates the pattern (and its scratch) stream-ordered on `stream` from
+ *   the library's own memory pool, and synchronises the stream once to learn
+ *   the CSR size.
+ *   Returns LOSA_ERR_ARG (null pointer, sizes, tau outside (0, 1]),
+ *   LOSA_ERR_MASS (a mass entry NaN, Inf, < 0 or >= 2), LOSA_ERR_NOMEM,
+ *   LOSA_ERR_CUDA.
+ */
+int losa_select(const float* mass, int B, int H, int n_blocks, int block, double tau,
+                losa_pattern** out, void* stream);
+
+/* Fills *view from a pattern. Returns LOSA_ERR_ARG on NULL. */
+int losa_pattern_info(const losa_pattern* p, losa_pattern_view* view);
+
+/*
+ * losa_pattern_export - copies the pattern's arrays into caller buffers
+ * (host or device memory; cudaMemcpyDefault) so a frozen pattern can be
+ * stored for reuse (ubos.tech LoSA post, Phase 2: the mask "is stored for
+ * reuse"). Any destination may be NULL to skip it; sizes are those of
+ * losa_pattern_view. The copies are ordered on `stream`; the call
+ * synchronises the stream before returning, so host buffers are filled.
+ */
+int losa_pattern_export(const losa_pattern* p, int32_t* row_ptr, int32_t* col_idx,
+                        int64_t* retained_fx, int64_t* total_fx, int32_t* tile_ptr,
+                        int32_t* tile_entry, int32_t* tile_order, void* stream);
+
+/*
+ * losa_sparse_attn - later steps: attention of fresh Q/K/V restricted to the
+ * frozen retained key blocks (Phase 3 - Repeated Sparse Inference, ubos.tech
+ * LoSA post; legiblepapers.com "Summary & Methodology Analysis").
+ *
+ *   q, k, v   [B, H, L_pad, d] device, L_pad = p->n_blocks * p->block.
+ *   o         [B, H, L_pad, d], out_dtype: for i in query block I,
+ *             O_i = sum_{j in R(I), j<L} softmax_j(scale q_i.k_j) v_j with the
+ *             softmax renormalised over the retained keys R(I) only.
+ *   lse       [B, H, L_pad] fp32, may be NULL: log-sum-exp over the retained keys.
+ *   Returns LOSA_ERR_ARG for a null pointer, a bad dtype, d not in {64, 128},
+ *   L < 1, L > L_pad or L_pad - L >= block.
+ */
+int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, int d,
+                     int L, float scale, const losa_pattern* p,
+                     void* o, int out_dtype, float* lse, void* stream);
+
+/* Frees a pattern. The memory returns to the library's pool in stream order
+ * on the stream the pattern was built on, so work on that stream that uses
+ * the pattern may still be in flight; work on OTHER streams that uses it must
+ * be complete (or ordered before that stream) first. NULL is a no-op. */
+void losa_free(losa_pattern* p);
+
+/*
+ * losa_check_status - synchronises `stream`, then reads and clears the
+ * device status word of the current device. Returns LOSA_ERR_TIMEOUT when a
+ * kernel since the last check gave up a bounded wait (its outputs are then
+ * undefined), else LOSA_OK or LOSA_ERR_CUDA.
+ */
+int losa_check_status(void* stream);
+
+/* Short English text for a status code. Never NULL. */
+const char* losa_strerror(int status);
+
+/* Library version, "major.minor.patch". */
+const char* losa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOSA_H_ */

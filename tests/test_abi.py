@@ -1,0 +1,103 @@
+"""The C-ABI library loads, exports every symbol include/losa.h declares, and
+rejects bad arguments on the host (no device work, so no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "losa.h")
+
+
+def _build():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "losa_build", os.path.join(ROOT, "block_sparse_attention_losa_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="module")
+def losa():
+    _build()
+    import block_sparse_attention_losa_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(losa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_method_calls():
+    names = declared_functions()
+    for n in ("losa_dense_mass", "losa_select", "losa_sparse_attn", "losa_free"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(losa):
+    lib = ctypes.CDLL(losa.LIB_PATH)
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    for n in names:
+        assert hasattr(lib, n), f"liblosa.so does not export {n}"
+    assert sorted(losa.EXPORTS) == names
+
+
+def test_strerror_and_version(losa):
+    lib = losa.lib()
+    assert lib.losa_strerror(0) == b"ok"
+    for code in range(-6, 0):
+        assert lib.losa_strerror(code) != b"unknown status"
+    assert lib.losa_strerror(-99) == b"unknown status"
+    assert re.fullmatch(rb"\d+\.\d+\.\d+", lib.losa_version())
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: the checks fail first
+
+
+def _dense(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, in_dt=0, B=1, H=2, L=250, L_pad=256, d=64, block=32,
+             scale=0.125, o=FAKE, out_dt=1, lse=FAKE, mass=FAKE, stream=None)
+    a.update(kw)
+    return lib.losa_dense_mass(a["q"], a["k"], a["v"], a["in_dt"], a["B"], a["H"], a["L"],
+                               a["L_pad"], a["d"], a["block"], a["scale"], a["o"], a["out_dt"],
+                               a["lse"], a["mass"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(q=None), dict(mass=None), dict(lse=None), dict(in_dt=7), dict(out_dt=-1),
+    dict(B=0), dict(H=0), dict(L=0), dict(L=300), dict(L_pad=250, L=250),
+    dict(L=200), dict(d=96), dict(block=16), dict(block=256), dict(scale=0.0),
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(L=70000, L_pad=70016, block=32),
+    dict(B=300, H=300), dict(q=ctypes.c_void_p(0x10008)),
+])
+def test_dense_mass_rejects_bad_arguments(losa, bad):
+    assert _dense(losa.lib(), **bad) == -1
+
+
+@pytest.mark.parametrize("tau", [0.0, -0.5, 1.0000001, 2.0, float("nan")])
+def test_select_rejects_tau_outside_unit_interval(losa, tau):
+    out = ctypes.c_void_p(123)
+    st = losa.lib().losa_select(FAKE, 1, 2, 8, 32, tau, ctypes.byref(out), None)
+    assert st == -1 and out.value is None
+
+
+@pytest.mark.parametrize("shape", [(0, 2, 8, 32), (1, 0, 8, 32), (1, 2, 0, 32),
+                                   (1, 2, 2048, 32), (1, 2, 8, 48)])
+def test_select_rejects_bad_shapes(losa, shape):
+    out = ctypes.c_void_p()
+    B, H, n, b = shape
+    assert losa.lib().losa_select(FAKE, B, H, n, b, 0.99, ctypes.byref(out), None) == -1
+
+
+def test_null_handles(losa):
+    lib = losa.lib()
+    view = losa.PatternView()
+    assert lib.losa_pattern_info(None, ctypes.byref(view)) == -1
+    assert lib.losa_sparse_attn(FAKE, FAKE, FAKE, 0, 64, 10, 0.1, None, FAKE, 1, None, None) == -1
+    assert lib.losa_pattern_export(None, None, None, None, None, None, None, None, None) == -1
+    lib.losa_free(None)  # no-op

@@ -1,0 +1,270 @@
+"""GPU path (through the C ABI) against the CPU oracle, element by element.
+
+Tolerances, per output:
+  * block mass: |delta| <= 1e-5 absolute (fp32 accumulation of exact
+    bf16 x bf16 products; the row sums to 1, so fp32 rounding of the sum
+    and of exp2 stays near 1e-7 per term).
+  * selection: bit-exact (row_ptr, col_idx, retained_fx, total_fx) against
+    the oracle's selection run on the GPU's own fp32 masses; with the
+    oracle's fp64 masses, the kept set still holds >= tau - 1e-5 of the mass.
+  * O (fp32 output): max |delta| <= 1e-2 and mean |delta| <= 1e-3 against
+    fp64 on the same bf16 inputs. P is rounded to bf16 before the P.V
+    product (relative 2^-9 per weight), which bounds the error near
+    2^-9 * max|v| ~ 0.008 in the worst case and ~1e-4 on average.
+  * O (bf16 output): additionally the output's own rounding, half an ulp:
+    |delta| <= 1e-2 + 2^-8 |O|.
+  * lse: |delta| <= 1e-4 (fp32 scores of exact products; the sum of exp
+    uses the unrounded fp32 values).
+"""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MASS_ATOL = 1e-5
+O_MAX, O_MEAN = 1e-2, 1e-3
+LSE_ATOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def losa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import block_sparse_attention_losa_b200 as m
+    return m
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def assert_o_close(o_gpu, o_ref, L, bf16_out=False, what="O"):
+    o = f64(o_gpu)
+    d = np.abs(o[:, :, :L] - o_ref[:, :, :L])
+    if bf16_out:
+        bound = O_MAX + 2.0 ** -8 * np.abs(o_ref[:, :, :L])
+        assert np.all(d <= bound), f"{what}: max excess {np.max(d - bound)}"
+    else:
+        assert d.max() <= O_MAX, f"{what}: max |d| {d.max()}"
+    assert d.mean() <= O_MEAN, f"{what}: mean |d| {d.mean()}"
+    assert np.all(o[:, :, L:] == 0), f"{what}: padded rows not zero"
+
+
+def assert_lse_close(lse_gpu, lse_ref, L):
+    l = f64(lse_gpu)
+    assert np.max(np.abs(l[:, :, :L] - lse_ref[:, :, :L])) <= LSE_ATOL
+    assert np.all(np.isneginf(l[:, :, L:]))
+
+
+def check_tiles(ex, pat, n):
+    """The sparse kernel's work list is the per-tile union of the rows'
+    kept sets, with correct masks, ordered by entry count (largest first)."""
+    row_ptr = ex["row_ptr"].numpy()
+    col_idx = ex["col_idx"].numpy()
+    tile_ptr = ex["tile_ptr"].numpy()
+    tile_entry = ex["tile_entry"].numpy()
+    order = ex["tile_order"].numpy()
+    qpt = 128 // pat.block
+    n_qt = (n * pat.block + 127) // 128
+    assert sorted(order.tolist()) == list(range(pat.n_tiles))
+    counts = np.diff(tile_ptr)
+    assert np.all(np.diff(counts[order]) <= 0)
+    for t in range(pat.n_tiles):
+        bh, qt = divmod(t, n_qt)
+        want = {}
+        for q in range(qpt):
+            I = qt * qpt + q
+            if I >= n:
+                break
+            r = bh * n + I
+            for J in col_idx[row_ptr[r]:row_ptr[r + 1]]:
+                want[int(J)] = want.get(int(J), 0) | (1 << q)
+        got = tile_entry[tile_ptr[t]:tile_ptr[t + 1]]
+        assert [int(e) & 0xFFFF for e in got] == sorted(want)
+        assert [int(e) >> 16 for e in got] == [want[J] for J in sorted(want)]
+
+
+def check_selection(pat, mass_gpu, tau, check_tile_lists=True):
+    mass_np = mass_gpu.cpu().numpy()
+    ref = O.select(mass_np, tau)
+    ex = {k: v.cpu() for k, v in pat.export("cpu").items()}
+    assert pat.nnz == len(ref["col_idx"])
+    np.testing.assert_array_equal(ex["row_ptr"].numpy(), ref["row_ptr"])
+    np.testing.assert_array_equal(ex["col_idx"].numpy(), ref["col_idx"])
+    assert ex["retained_fx"].tolist() == ref["retained_fx"]
+    assert ex["total_fx"].tolist() == ref["total_fx"]
+    if check_tile_lists:
+        check_tiles(ex, pat, mass_np.shape[-1])
+    return ref, ex
+
+
+def run_small(losa, wl, tau=0.99, out_dtype=torch.float32, in_fp32=None):
+    q, k, v = W.generate(wl, dtype=torch.float32)
+    if in_fp32 is None:
+        in_fp32 = wl.in_dtype == "fp32"
+    dt = torch.float32 if in_fp32 else torch.bfloat16
+    qd, kd, vd = (t.to("cuda", dt) for t in (q, k, v))
+    L, b, scale = wl.seq_len, wl.block, 1 / math.sqrt(wl.head_dim)
+    o, lse, mass = losa.dense_mass(qd, kd, vd, L, b, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    losa.check_status()
+    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
+    o_ref, lse_ref = O.dense_attention(q64, k64, v64, L, scale)
+    mass_ref = O.block_mass(q64, k64, L, b, scale)
+    assert_o_close(o, o_ref, L, bf16_out=out_dtype == torch.bfloat16, what="dense O")
+    assert_lse_close(lse, lse_ref, L)
+    m = f64(mass)
+    assert np.max(np.abs(m - mass_ref)) <= MASS_ATOL, np.max(np.abs(m - mass_ref))
+
+    pat = losa.select(mass, b, tau)
+    ref, ex = check_selection(pat, mass, tau)
+    # Against the oracle's own fp64 masses the kept set still reaches tau.
+    for r in range(pat.rows):
+        bb, rest = divmod(r, wl.heads * wl.n_blocks)
+        h, I = divmod(rest, wl.n_blocks)
+        cols = ex["col_idx"][ex["row_ptr"][r]:ex["row_ptr"][r + 1]].numpy()
+        assert mass_ref[bb, h, I, cols].sum() >= tau - 1e-5
+
+    q2, k2, v2 = W.drift(wl, (q, k, v), step=1, dtype=torch.float32)
+    q2d, k2d, v2d = (t.to("cuda", dt) for t in (q2, k2, v2))
+    o2, lse2 = losa.sparse_attn(q2d, k2d, v2d, L, pat, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    losa.check_status()
+    o2_ref, lse2_ref = O.sparse_attention(q2.double().numpy(), k2.double().numpy(),
+                                          v2.double().numpy(), L, b, scale, ref["row_ptr"],
+                                          ref["col_idx"])
+    assert_o_close(o2, o2_ref, L, bf16_out=out_dtype == torch.bfloat16, what="sparse O")
+    assert_lse_close(lse2, lse2_ref, L)
+    return pat
+
+
+def test_tiny_workload(losa):
+    pat = run_small(losa, W.WORKLOADS["tiny"])
+    assert 0.3 <= 1 - pat.density() <= 0.5
+
+
+SMALL = [
+    # name, heads, d, grid, block, text, batch — ragged tails and partial tiles
+    ("d128_b64_partial_tile", 3, 128, (3, 10, 13), 64, 0, 1),
+    ("d64_b128_text", 2, 64, (2, 12, 20), 128, 30, 1),
+    ("d128_b32_partial_tile", 2, 128, (3, 7, 9), 32, 0, 1),
+    ("d64_b64_text", 2, 64, (4, 9, 11), 64, 20, 1),
+    ("d128_b64_batch2", 2, 128, (2, 8, 16), 64, 0, 2),
+    ("d128_b128_10_blocks", 2, 128, (4, 16, 20), 128, 0, 1),
+    ("d64_b32_exact", 1, 64, (2, 8, 8), 32, 0, 1),
+]
+
+
+@pytest.mark.parametrize("name,heads,d,grid,block,text,batch", SMALL, ids=[s[0] for s in SMALL])
+def test_small_shapes(losa, name, heads, d, grid, block, text, batch):
+    wl = W.custom(name, heads, d, grid, block, text_tokens=text, batch=batch, amplitude=1.2,
+                  seed=zlib.crc32(name.encode()) % 1000)
+    run_small(losa, wl)
+
+
+@pytest.mark.parametrize("tau", [0.5, 0.95, 0.999])
+def test_tau_values(losa, tau):
+    wl = W.custom("tau", 2, 128, (3, 10, 13), 64, amplitude=1.2, seed=5)
+    run_small(losa, wl, tau=tau)
+
+
+def test_bf16_io(losa):
+    wl = W.custom("bf16io", 2, 128, (3, 10, 13), 64, amplitude=1.2, seed=9)
+    run_small(losa, wl, out_dtype=torch.bfloat16, in_fp32=False)
+
+
+def test_fp32_inputs_are_rounded_to_bf16(losa):
+    wl = W.custom("fp32in", 2, 64, (3, 10, 13), 64, amplitude=1.2, seed=11, in_dtype="fp32")
+    run_small(losa, wl, in_fp32=True)
+
+
+def test_tau_one_keeps_every_positive_block_and_equals_dense(losa):
+    wl = W.custom("tau1", 2, 64, (2, 8, 16), 32, amplitude=0.8, seed=3)
+    q, k, v = (t.cuda() for t in W.generate(wl, dtype=torch.bfloat16))
+    L, b = wl.seq_len, wl.block
+    o, lse, mass = losa.dense_mass(q, k, v, L, b)
+    pat = losa.select(mass, b, 1.0)
+    x = O.to_fixed(mass.cpu().numpy())
+    assert pat.nnz == int((x > 0).sum())
+    o2, lse2 = losa.sparse_attn(q, k, v, L, pat)
+    torch.cuda.synchronize()
+    if pat.nnz == pat.rows * pat.n_blocks:
+        # every block kept: the sparse kernel computes the dense result
+        q64, k64, v64 = (t.double().cpu().numpy() for t in (q, k, v))
+        o_ref, lse_ref = O.dense_attention(q64, k64, v64, L, 1 / math.sqrt(wl.head_dim))
+        assert_o_close(o2, o_ref, L, what="tau=1 sparse O")
+        assert_lse_close(lse2, lse_ref, L)
+
+
+def test_one_hot_mass_rows_keep_one_block(losa):
+    """A mass map with one block per row at mass 1 keeps exactly that block."""
+    n = 40
+    mass = torch.zeros(1, 3, n, n)
+    rng = np.random.default_rng(0)
+    hot = rng.integers(0, n, size=(3, n))
+    for h in range(3):
+        for I in range(n):
+            mass[0, h, I, hot[h, I]] = 1.0
+    pat = losa.select(mass.cuda(), 64, 0.99)
+    ex = pat.export("cpu")
+    assert pat.nnz == 3 * n
+    assert ex["col_idx"].numpy().tolist() == hot.reshape(-1).tolist()
+
+
+def test_equal_masses_break_ties_by_lower_index(losa):
+    n = 16
+    mass = torch.full((1, 1, n, n), 1.0 / n)
+    pat = losa.select(mass.cuda(), 32, 0.5)
+    ex = pat.export("cpu")
+    assert ex["col_idx"].numpy().tolist() == list(range(8)) * n
+
+
+def test_random_mass_maps_select_bit_exact(losa):
+    """Selection alone on random and adversarial mass maps (many ties,
+    zeros, tiny values), against the oracle."""
+    rng = np.random.default_rng(7)
+    for trial in range(6):
+        n = int(rng.choice([8, 33, 129, 500, 2047]))
+        H = 2 if n <= 500 else 1
+        if trial % 3 == 0:
+            m = rng.integers(0, 5, size=(1, H, n, n)).astype(np.float32)
+        elif trial % 3 == 1:
+            m = (rng.random((1, H, n, n)) ** 8).astype(np.float32)
+        else:
+            m = rng.dirichlet(np.ones(n) * 0.1, size=(1, H, n)).astype(np.float32)
+        m /= np.maximum(m.sum(axis=-1, keepdims=True), 1e-30)
+        m = m.astype(np.float32)
+        for tau in (0.3, 0.99, 1.0):
+            t = torch.from_numpy(m).cuda()
+            pat = losa.select(t, 64, tau)
+            check_selection(pat, t, tau, check_tile_lists=(n <= 129))
+
+
+def test_bad_mass_is_reported(losa):
+    mass = torch.full((1, 1, 8, 8), 0.125)
+    mass[0, 0, 3, 5] = float("nan")
+    with pytest.raises(losa.LosaError) as e:
+        losa.select(mass.cuda(), 32, 0.99)
+    assert e.value.status == -5
+    mass[0, 0, 3, 5] = -0.1
+    with pytest.raises(losa.LosaError):
+        losa.select(mass.cuda(), 32, 0.99)
+    # the status word was cleared: a good map goes through
+    mass[0, 0, 3, 5] = 0.125
+    losa.select(mass.cuda(), 32, 0.99)
+
+
+def test_shape_mismatch_is_rejected(losa):
+    wl = W.custom("mm", 1, 64, (2, 8, 8), 32, amplitude=1.0, seed=1)
+    q, k, v = (t.cuda() for t in W.generate(wl, dtype=torch.bfloat16))
+    _, _, mass = losa.dense_mass(q, k, v, wl.seq_len, wl.block)
+    pat = losa.select(mass, wl.block, 0.99)
+    q2 = torch.zeros(1, 1, 256 + 32, 64, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        losa.sparse_attn(q2, q2, q2, wl.seq_len, pat)
