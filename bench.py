@@ -74,6 +74,29 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def attention_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("losa_attention.cuh", "losa_device.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_losa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload):
+    """Per-launch DRAM bytes of the sparse kernel from the committed ncu
+    summary, or None if the kernel sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", f"traffic_sparse_attn_{workload}.txt")
+    try:
+        kv = dict(line.split(None, 1) for line in open(path)
+                  if line.strip() and not line.startswith("#"))
+    except OSError:
+        return None
+    if kv.get("source_sha", "").strip() != attention_source_sha():
+        return None
+    return float(kv["dram_read_bytes"]) + float(kv["dram_write_bytes"])
+
+
 def step_flops(wl, nnz, n_sparse):
     """Algorithmic FLOPs of one step: construction pass + sparse steps."""
     B, H, Lp, d, b = wl.batch, wl.heads, wl.seq_pad, wl.head_dim, wl.block
@@ -374,7 +397,8 @@ def main():
         "sparse_vs_dense_speedup": (dense_ms * 4.0 / 6.0) / sparse_ms,
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": sparse_tf,
                      "peak": peak, "unit": "TFLOP/s", "frac": sparse_tf / peak,
-                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                     "traffic": measured_traffic(wl.name),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
         "gpu_launches": args.steps * (LAUNCHES_DENSE + LAUNCHES_SELECT + n_sparse * LAUNCHES_SPARSE),
         "clocks": clock_info,
     }
