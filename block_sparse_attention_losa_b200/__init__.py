@@ -28,8 +28,9 @@ STATUS = {0: "LOSA_OK", -1: "LOSA_ERR_ARG", -2: "LOSA_ERR_CUDA", -3: "LOSA_ERR_N
 
 # Every symbol include/losa.h declares.
 EXPORTS = ("losa_dense_mass", "losa_select", "losa_pattern_info", "losa_pattern_export",
-           "losa_sparse_attn", "losa_free", "losa_check_status", "losa_strerror",
-           "losa_version")
+           "losa_select_noalloc", "losa_sparse_attn", "losa_free", "losa_check_status",
+           "losa_strerror", "losa_version")
+NOALLOC_MAX_ROWS = 65536  # LOSA_NOALLOC_MAX_ROWS
 
 
 class LosaError(RuntimeError):
@@ -64,6 +65,9 @@ def _load():
     lib.losa_pattern_info.restype = i32
     lib.losa_pattern_export.argtypes = [vp] * 9
     lib.losa_pattern_export.restype = i32
+    i64 = ctypes.c_int64
+    lib.losa_select_noalloc.argtypes = [vp, i32, i32, i32, f64, vp, vp, i64, vp, vp, vp]
+    lib.losa_select_noalloc.restype = i32
     lib.losa_sparse_attn.argtypes = [vp, vp, vp, i32, i32, i32, f32, vp, vp, i32, vp, vp]
     lib.losa_sparse_attn.restype = i32
     lib.losa_free.argtypes = [vp]

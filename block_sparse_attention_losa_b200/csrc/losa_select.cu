@@ -17,6 +17,7 @@
 #include <cub/block/block_scan.cuh>
 
 #include <cstdio>
+#include <mutex>
 #include <vector>
 
 #include "losa_device.cuh"
@@ -398,3 +399,97 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
 }
 
 }  // namespace losa
+
+// ---------------------------------------------------------------------------
+// Allocation-free selection (losa_select_noalloc): the cut and count kernels
+// above, with their per-row scratch in a fixed device array instead of
+// stream-ordered allocations, and the kept lists written straight into the
+// caller's CSR buffers.
+
+namespace losa {
+namespace {
+
+constexpr int kNoallocMaxRows = LOSA_NOALLOC_MAX_ROWS;
+constexpr size_t kNoallocCutBytes = size_t(kNoallocMaxRows) * 8;
+constexpr size_t kNoallocBytes = kNoallocCutBytes + size_t(kNoallocMaxRows) * 4;
+
+// Per-row cut keys, then per-row kept counts. Every element a call reads is
+// written earlier in the same call, so nothing needs clearing between calls.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side name is not a device address).
+unsigned char* noalloc_scratch() {
+  constexpr int kMaxDevices = 64;
+  static unsigned char* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  return addr[dev];
+}
+
+// One CTA per row: the row's kept key blocks, ascending, at row_ptr[row].
+__global__ void __launch_bounds__(kSelThreads)
+    row_write_kernel(const float* __restrict__ mass, int n,
+                     const unsigned long long* __restrict__ cut_key,
+                     const int* __restrict__ row_ptr, int* __restrict__ col_idx,
+                     long long capacity) {
+  using Scan = cub::BlockScan<int, kSelThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  const int row = blockIdx.x;
+  const unsigned long long cut = cut_key[row];
+  long long base = row_ptr[row];
+  for (int c0 = 0; c0 < n; c0 += kSelThreads) {
+    const int J = c0 + threadIdx.x;
+    int keep = 0;
+    if (J < n) {
+      long long x;
+      to_fixed(mass[size_t(row) * n + J], x);
+      keep = sort_key(x, J) <= cut;
+    }
+    int ex, tot;
+    Scan(tmp).ExclusiveSum(keep, ex, tot);
+    __syncthreads();
+    if (keep && base + ex < capacity) col_idx[base + ex] = J;
+    base += tot;
+  }
+}
+
+}  // namespace
+}  // namespace losa
+
+extern "C" int losa_select_noalloc(const float* mass, int B, int H, int n_blocks, double tau,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   int64_t* retained_fx, int64_t* total_fx, void* stream) {
+  using namespace losa;
+  if (!mass || !row_ptr || !col_idx || !retained_fx || !total_fx) return LOSA_ERR_ARG;
+  if (B < 1 || H < 1 || n_blocks < 1 || n_blocks > 2047) return LOSA_ERR_ARG;
+  const int64_t R = int64_t(B) * H * n_blocks;
+  if (R > kNoallocMaxRows) return LOSA_ERR_ARG;
+  if (!(tau > 0.0 && tau <= 1.0) || col_capacity < 0) return LOSA_ERR_ARG;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return LOSA_ERR_CUDA;
+  if (major != 10) return LOSA_ERR_UNSUPPORTED;
+  unsigned char* scratch = noalloc_scratch();
+  int* status = device_status_word();
+  if (!scratch || !status) return LOSA_ERR_CUDA;
+  auto* cut = reinterpret_cast<unsigned long long*>(scratch);
+  auto* cnt = reinterpret_cast<int*>(scratch + kNoallocCutBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned long long tau_fx = (unsigned long long)llrint(tau * 281474976710656.0);
+  select_cut_kernel<<<unsigned(R), kSelThreads, 0, s>>>(mass, n_blocks, tau_fx, cut, cnt,
+                                                         (long long*)retained_fx,
+                                                         (long long*)total_fx, status);
+  scan_kernel<<<1, 1024, 0, s>>>(cnt, int(R), row_ptr);
+  row_write_kernel<<<unsigned(R), kSelThreads, 0, s>>>(mass, n_blocks, cut, row_ptr, col_idx,
+                                                       (long long)col_capacity);
+  return cudaGetLastError() == cudaSuccess ? LOSA_OK : LOSA_ERR_CUDA;
+}

@@ -175,6 +175,43 @@ int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, 
                      int L, float scale, const losa_pattern* p,
                      void* o, int out_dtype, float* lse, void* stream);
 
+/* Largest B*H*n_blocks that losa_select_noalloc accepts. */
+#define LOSA_NOALLOC_MAX_ROWS 65536
+
+/*
+ * losa_select_noalloc - the same selection as losa_select, for callers that
+ * cannot allocate device memory, written straight into buffers the caller
+ * owns. The LoSA pages have no counterpart to this call; it exists for
+ * callers such as serving engines that reserve all device memory at
+ * start-up and forbid allocation while requests run, code that lives inside
+ * another framework's allocator, and latency-critical loops that cannot
+ * afford cudaMalloc's implicit device synchronisation.
+ *
+ *   mass         [B, H, n, n] fp32 device.
+ *   row_ptr      [R + 1] int32 device, R = B*H*n: CSR row offsets
+ *                (row_ptr[R] = number of kept blocks).
+ *   col_idx      [col_capacity] int32 device: kept key blocks, ascending
+ *                per row. Entries at offsets >= col_capacity are dropped;
+ *                col_capacity >= R*n always suffices. Compare row_ptr[R]
+ *                with col_capacity to see whether everything fit.
+ *   retained_fx, total_fx  [R] int64 device, as in losa_pattern_view.
+ *
+ * It allocates nothing: its scratch (one 64-bit cut key and one count per
+ * row, 768 KB in all) is a fixed array inside the library that every GPU
+ * which loads the library holds until the process exits. Hence R must not
+ * exceed LOSA_NOALLOC_MAX_ROWS (LOSA_ERR_ARG otherwise). Every call shares
+ * that array, so calls that overlap on the GPU (on different streams, or
+ * from different threads) race and must be serialised by the caller. The
+ * first call on a device looks up the array's device address; make that
+ * first call before any stream capture. The call does not synchronise: a
+ * bad mass value is reported by the next losa_check_status.
+ * Returns LOSA_OK, LOSA_ERR_ARG (null pointer, sizes, tau outside (0, 1],
+ * col_capacity < 0), LOSA_ERR_UNSUPPORTED or LOSA_ERR_CUDA.
+ */
+int losa_select_noalloc(const float* mass, int B, int H, int n_blocks, double tau,
+                        int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                        int64_t* retained_fx, int64_t* total_fx, void* stream);
+
 /* Frees a pattern. The memory returns to the library's pool in stream order
  * on the stream the pattern was built on, so work on that stream that uses
  * the pattern may still be in flight; work on OTHER streams that uses it must
