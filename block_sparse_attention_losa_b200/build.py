@@ -44,17 +44,35 @@ def build(force: bool = False, verbose: bool = False) -> str:
     out_tmp = LIB + ".tmp"
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
            "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"), "-o", out_tmp]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
+           "-Xptxas", "-v", "-I", os.path.join(ROOT, "include"), "-o", out_tmp]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stderr)
+    check_attention_registers(res.stderr)
     os.replace(out_tmp, LIB)
     return LIB
+
+
+def check_attention_registers(ptxas_log: str, want: int = 168) -> None:
+    """The attention kernels split their launch registers between
+    warpgroups with setmaxnreg; the split adds up only if every instance
+    launches with exactly `want` registers per thread (else a warpgroup
+    would wait for registers that never come). Refuse the build otherwise."""
+    current, seen = None, 0
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            current = "attn_kernel" in line
+        elif current and "Used" in line and "registers" in line:
+            used = int(line.split("Used")[1].split("registers")[0])
+            seen += 1
+            if used != want:
+                raise RuntimeError(f"attention kernel launches with {used} registers, "
+                                   f"the setmaxnreg split assumes {want}")
+    if seen == 0:
+        raise RuntimeError("no attention kernel found in the ptxas log")
 
 
 if __name__ == "__main__":

@@ -57,7 +57,7 @@ cudaError_t run(const void* q, const void* k, const void* v, int BH, const AttnP
   if (!make_map(&tq, q, BH, p.L_pad, D, 128) || !make_map(&tk, k, BH, p.L_pad, D, BN) ||
       !make_map(&tv, v, BH, p.L_pad, D, BN))
     return cudaErrorInvalidValue;
-  kern<<<grid, 192, Lay::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  kern<<<grid, kAttnThreads, Lay::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -100,13 +100,13 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, in
   p.mass = mass;
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
-  const dim3 grid(p.n_qt, BH);
+  const dim3 grid((p.n_qt + 1) / 2, BH);  // two query tiles per CTA
   if (d == 128) {
     return out_bf16 ? run<128, 128, 2, true, true>(q, k, v, BH, p, grid, stream)
                     : run<128, 128, 2, true, false>(q, k, v, BH, p, grid, stream);
   }
-  return out_bf16 ? run<64, 128, 3, true, true>(q, k, v, BH, p, grid, stream)
-                  : run<64, 128, 3, true, false>(q, k, v, BH, p, grid, stream);
+  return out_bf16 ? run<64, 128, 4, true, true>(q, k, v, BH, p, grid, stream)
+                  : run<64, 128, 4, true, false>(q, k, v, BH, p, grid, stream);
 }
 
 cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, int L,
@@ -129,7 +129,8 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, in
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
   const int BH = pat->B * pat->H;
-  const dim3 grid(unsigned(pat->n_tiles));
+  p.n_tiles = int(pat->n_tiles);
+  const dim3 grid(unsigned((pat->n_tiles + 1) / 2));  // two tiles per CTA
   if (pat->n_tiles == 0) return cudaSuccess;
 #define LOSA_SPARSE_CASE(D_, BN_, NS_)                                                    \
   if (d == D_ && pat->block == BN_)                                                      \
@@ -137,10 +138,10 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, in
                     : run<D_, BN_, NS_, false, false>(q, k, v, BH, p, grid, stream);
   LOSA_SPARSE_CASE(128, 128, 2)
   LOSA_SPARSE_CASE(128, 64, 4)
-  LOSA_SPARSE_CASE(128, 32, 4)
-  LOSA_SPARSE_CASE(64, 128, 3)
-  LOSA_SPARSE_CASE(64, 64, 4)
-  LOSA_SPARSE_CASE(64, 32, 4)
+  LOSA_SPARSE_CASE(128, 32, 8)
+  LOSA_SPARSE_CASE(64, 128, 4)
+  LOSA_SPARSE_CASE(64, 64, 8)
+  LOSA_SPARSE_CASE(64, 32, 8)
 #undef LOSA_SPARSE_CASE
   return cudaErrorInvalidValue;
 }

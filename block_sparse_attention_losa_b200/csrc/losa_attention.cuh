@@ -1,22 +1,33 @@
 // losa_attention.cuh - the attention kernels of the LoSA hot path (sm_100a).
 //
-// One CTA owns a 128-row query tile of one (batch, head) and walks a list of
-// key tiles. Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r of the tile (TMEM lane r);
-//   warp 4     TMA producer: Q once, then K (and V) tiles into smem rings;
-//   warp 5     MMA issuer (one thread) and TMEM owner.
-// Per key tile: S = Q K^T (tcgen05, bf16 -> fp32 in TMEM, double-buffered),
-// the softmax warps read S from TMEM, write P (bf16) into a 128B-swizzled
-// smem tile, and the MMA thread accumulates O += P V into TMEM.
+// One CTA owns two 128-row query tiles and walks, for each, a list of key
+// tiles. Warp roles (384 threads, three warpgroups):
+//   warps 0-3  softmax of tile 0 (thread r owns query row r = TMEM lane r),
+//   warps 4-7  softmax of tile 1,
+//   warp 8     TMA producer: Q tiles, then K and V tiles through smem rings,
+//   warp 9     MMA issuer (one thread) and TMEM owner,
+//   warps 10-11 idle.
+// The kernel launches with 168 registers per thread (384 x 168 = 64,512);
+// the third warpgroup gives registers back (setmaxnreg to 40) and the two
+// softmax warpgroups take them (to 232): 2*128*232 + 128*40 = 64,512.
+// TMEM (512 columns): S_t at columns [128 t, 128 t + BN), O_t at 256 + t D.
+// Per key tile j of tile t: S_t = Q_t K_j^T (tcgen05 kind::f16, bf16 operands
+// from 128B-swizzled smem, fp32 in TMEM); the softmax warps read S_t, write
+// the bf16 weights P_t back over the first BN/2 columns of S_t, and the MMA
+// thread accumulates O_t += P_t V_j with P_t read straight from TMEM. The MMA
+// thread interleaves the two tiles - PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) -
+// so the tensor core works on one tile while the other tile's softmax runs.
 //
-// kDense = true is the construction step: pass 1 is the flash forward over
-// all key tiles (O, row lse); pass 2 recomputes S = Q K^T tile by tile and
-// sums exp(s - lse) over each (query block, key block) into the mass map
-// (LoSA abstract, arXiv 2608.12032: exact block attention masses at one
-// early dense step; ubos.tech LoSA post, Phase 1 - Dense Calibration).
-// kDense = false is the sparse step: pass 1 only, over the tile's union of
-// retained key blocks, each row masked to its own query block's set
-// (ubos.tech LoSA post, Phase 3 - Repeated Sparse Inference).
+// kDense = true is the construction step: both tiles are adjacent query tiles
+// of one head and share every K/V tile. Pass 1 is the flash forward over all
+// key tiles (O, row lse); pass 2 recomputes S = Q K^T tile by tile and sums
+// exp(s - lse) over each (query block, key block) straight into the mass map
+// (LoSA abstract, arXiv 2608.12032: exact block attention masses at one early
+// dense step; ubos.tech LoSA post, Phase 1 - Dense Calibration).
+// kDense = false is the sparse step: the two tiles are independent work
+// items with their own lists (the union of their query blocks' retained key
+// blocks), each row masked to its own query block's set (ubos.tech LoSA
+// post, Phase 3 - Repeated Sparse Inference).
 #pragma once
 
 #include "losa_device.cuh"
@@ -28,6 +39,7 @@ struct AttnParams {
   int L_pad;      // padded tokens (multiple of block)
   int n_qt;       // query tiles per head = ceil(L_pad / 128)
   int n_kv;       // key tiles per pass (dense)
+  int n_tiles;    // sparse: number of tiles in tile_order
   int block;      // LoSA block size b
   int n_blocks;   // L_pad / block
   float scale_log2;  // softmax scale * log2(e)
@@ -43,35 +55,41 @@ struct AttnParams {
 template <int D, int BN, int NS>
 struct AttnLayout {
   static constexpr int BM = 128;
-  static constexpr int kSlab = 64;                       // bf16 elements per 128 B row
-  static constexpr int Q_BYTES = BM * D * 2;             // D/64 slabs of 16 KB
+  static constexpr int NT = 2;                           // query tiles per CTA
+  static constexpr int Q_BYTES = BM * D * 2;             // one tile: D/64 slabs of 16 KB
   static constexpr int KV_BYTES = BN * D * 2;            // D/64 slabs of BN*128 B
-  static constexpr int P_SLABS = (BN + 63) / 64;
-  static constexpr int P_BYTES = P_SLABS * BM * 128;     // 128 rows x 128 B per slab
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int N_BARS = 1 + 4 * NS + 9;
+  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  // q_full[2], k_full/k_empty/v_full/v_empty[NS], s_full[2], s_free[2],
+  // p_full[2], o_full[2], red_bar[2][2], drain
+  static constexpr int N_BARS = 2 + 4 * NS + 8 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem addr, abort flag
-  static constexpr int OFF_RED = OFF_MISC + 16;          // float red[2][4][4]
-  static constexpr int BYTES = OFF_RED + 2 * 4 * 4 * 4;
-  static constexpr int SMEM_ALLOC = BYTES + 1024;        // slack for 1 KB alignment
-  static constexpr int TMEM_NEED = 2 * BN + D;
-  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
-                                 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int TMEM_O = 2 * BN;
-  static_assert(D % 64 == 0, "head dim must be a multiple of 64");
+  static constexpr int OFF_RED = OFF_MISC + 16;          // float red[2 tiles][2][4 warps][4]
+  static constexpr int BYTES = OFF_RED + 2 * 2 * 4 * 4 * 4;
+  // Slack for 1 KB alignment; never below 120 KB, so that two CTAs cannot
+  // share an SM (each CTA allocates all 512 TMEM columns).
+  static constexpr int SMEM_ALLOC = BYTES + 1024 > 120 * 1024 ? BYTES + 1024 : 120 * 1024;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
+  static_assert(D % 64 == 0 && D <= 128, "head dim must be 64 or 128");
   static_assert(BN % 32 == 0 && BN <= 128, "key tile must be 32, 64 or 128");
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0, "1 KB alignment");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "1 KB alignment");
   static_assert(KV_BYTES % 1024 == 0, "1 KB alignment of stages");
-  // More than half of TMEM per CTA is only safe with one CTA per SM.
-  static_assert(TMEM_COLS <= 256 || SMEM_ALLOC > 116 * 1024, "TMEM oversubscription");
+  static_assert(SMEM_ALLOC > 116 * 1024, "all of TMEM per CTA needs one CTA per SM");
+  static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
 };
 
+constexpr int kAttnThreads = 384;
+constexpr int kAttnLaunchRegs = 168;   // checked against ptxas at build time
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kAttnThreads * kAttnLaunchRegs,
+              "register split must use exactly the launch allocation");
+
 template <int D, int BN, int NS, bool kDense, bool kOutBf16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using Lay = AttnLayout<D, BN, NS>;
@@ -86,167 +104,264 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = smem + Lay::OFF_Q;
   uint8_t* sK = smem + Lay::OFF_K;
   uint8_t* sV = smem + Lay::OFF_V;
-  uint8_t* sP = smem + Lay::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + NS;
-  uint64_t* v_full = k_empty + NS;
-  uint64_t* v_empty = v_full + NS;
-  uint64_t* s_full = v_empty + NS;  // [2]
-  uint64_t* s_free = s_full + 2;    // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* red_bar = pv_done + 1;  // [2], cross-warp mass reduction
-  uint64_t* drain_bar = red_bar + 2;  // MMA drain after an abort
+  uint64_t* q_full = bars;             // [2]
+  uint64_t* k_full = q_full + 2;       // [NS]
+  uint64_t* k_empty = k_full + NS;     // [NS]
+  uint64_t* v_full = k_empty + NS;     // [NS]
+  uint64_t* v_empty = v_full + NS;     // [NS]
+  uint64_t* s_full = v_empty + NS;     // [2] MMA -> softmax t: S_t ready
+  uint64_t* s_free = s_full + 2;       // [2] softmax t -> MMA: S_t read (pass 2)
+  uint64_t* p_full = s_free + 2;       // [2] softmax t -> MMA: P_t in TMEM
+  uint64_t* o_full = p_full + 2;       // [2] MMA -> softmax t: last PV_t done
+  uint64_t* red_bar = o_full + 2;      // [2][2] softmax t: mass reduction
+  uint64_t* drain_bar = red_bar + 4;   // MMA drain after an abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
-  float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);  // [2][4][4]
+  float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item
-  int bh, qt, e_begin = 0, n_iter;
+  // ---- work items: per tile t, its head, query tile and key list
+  int bh[2], qt[2], e_begin[2] = {0, 0}, n_it[2];
   if constexpr (kDense) {
-    qt = blockIdx.x;
-    bh = blockIdx.y;
-    n_iter = p.n_kv;
+    bh[0] = bh[1] = blockIdx.y;
+    qt[0] = 2 * blockIdx.x;
+    qt[1] = 2 * blockIdx.x + 1;  // may lie past the head: rows read as 0, nothing stored
+    n_it[0] = n_it[1] = p.n_kv;
   } else {
-    const int t = p.tile_order[blockIdx.x];
-    bh = t / p.n_qt;
-    qt = t - bh * p.n_qt;
-    e_begin = p.tile_ptr[t];
-    n_iter = p.tile_ptr[t + 1] - e_begin;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int idx = 2 * blockIdx.x + t;
+      if (idx < p.n_tiles) {
+        const int tile = p.tile_order[idx];
+        bh[t] = tile / p.n_qt;
+        qt[t] = tile - bh[t] * p.n_qt;
+        e_begin[t] = p.tile_ptr[tile];
+        n_it[t] = p.tile_ptr[tile + 1] - e_begin[t];
+      } else {
+        bh[t] = 0;
+        qt[t] = 0;
+        n_it[t] = 0;
+      }
+    }
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+      mbar_init(&red_bar[2 * t], 128);
+      mbar_init(&red_bar[2 * t + 1], 128);
+    }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
-    }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
-    mbar_init(&red_bar[0], 128);
-    mbar_init(&red_bar[1], 128);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc(tmem_slot, Lay::TMEM_COLS);
+  if (warp == 9) tmem_alloc(tmem_slot, Lay::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.status};
 
-  if (warp == 4) {
+  if (warp >= 8) {
+  reg_dealloc<kControlRegs>();
+  if (warp == 8) {
     // ================================================================ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      mbar_arrive_expect_tx(q_full, Lay::Q_BYTES);
 #pragma unroll
-      for (int s = 0; s < N_SLABS; ++s)
-        tma_load_3d(sQ + s * (BM * 128), &tm_q, q_full, s * 64, qt * BM, bh);
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(&q_full[t], Lay::Q_BYTES);
+#pragma unroll
+        for (int s = 0; s < N_SLABS; ++s)
+          tma_load_3d(sQ + t * Lay::Q_BYTES + s * (BM * 128), &tm_q, &q_full[t], s * 64,
+                      qt[t] * BM, bh[t]);
+      }
       int kc = 0, vc = 0;
       bool ok = true;
-      constexpr int n_pass = kDense ? 2 : 1;
-      for (int pass = 0; pass < n_pass && ok; ++pass) {
-        for (int it = 0; it < n_iter; ++it) {
-          int key_row;
-          if constexpr (kDense) {
-            key_row = it * BN;
-          } else {
-            key_row = (p.tile_entry[e_begin + it] & 0xFFFF) * BN;
-          }
-          const int ks = kc % NS;
-          if (!mbar_wait(&k_empty[ks], ((kc / NS) & 1) ^ 1, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[ks], Lay::KV_BYTES);
+      auto load_k = [&](int key_row, int head) -> bool {
+        const int ks = kc % NS;
+        if (!mbar_wait(&k_empty[ks], ((kc / NS) & 1) ^ 1, wc)) return false;
+        mbar_arrive_expect_tx(&k_full[ks], Lay::KV_BYTES);
 #pragma unroll
-          for (int s = 0; s < N_SLABS; ++s)
-            tma_load_3d(sK + ks * Lay::KV_BYTES + s * (BN * 128), &tm_k, &k_full[ks], s * 64,
-                        key_row, bh);
-          ++kc;
-          if (pass == 0) {
-            const int vs = vc % NS;
-            if (!mbar_wait(&v_empty[vs], ((vc / NS) & 1) ^ 1, wc)) { ok = false; break; }
-            mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
+        for (int s = 0; s < N_SLABS; ++s)
+          tma_load_3d(sK + ks * Lay::KV_BYTES + s * (BN * 128), &tm_k, &k_full[ks], s * 64,
+                      key_row, head);
+        ++kc;
+        return true;
+      };
+      auto load_v = [&](int key_row, int head) -> bool {
+        const int vs = vc % NS;
+        if (!mbar_wait(&v_empty[vs], ((vc / NS) & 1) ^ 1, wc)) return false;
+        mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
 #pragma unroll
-            for (int s = 0; s < N_SLABS; ++s)
-              tma_load_3d(sV + vs * Lay::KV_BYTES + s * (BN * 128), &tm_v, &v_full[vs], s * 64,
-                          key_row, bh);
-            ++vc;
+        for (int s = 0; s < N_SLABS; ++s)
+          tma_load_3d(sV + vs * Lay::KV_BYTES + s * (BN * 128), &tm_v, &v_full[vs], s * 64,
+                      key_row, head);
+        ++vc;
+        return true;
+      };
+      if constexpr (kDense) {
+        for (int j = 0; ok && j < p.n_kv; ++j) ok = load_k(j * BN, bh[0]) && load_v(j * BN, bh[0]);
+        for (int j = 0; ok && j < p.n_kv; ++j) ok = load_k(j * BN, bh[0]);
+      } else {
+        const int n_max = max(n_it[0], n_it[1]);
+        for (int j = 0; ok && j < n_max; ++j) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (ok && j < n_it[t]) {
+              const int row = (p.tile_entry[e_begin[t] + j] & 0xFFFF) * BN;
+              ok = load_k(row, bh[t]) && load_v(row, bh[t]);
+            }
           }
         }
       }
       if (!ok) {
         // Aborted: wait (bounded) for the copies still in flight before the
         // CTA releases its shared memory.
-        mbar_wait_drain(q_full, 0);
+        mbar_wait_drain(&q_full[0], 0);
+        mbar_wait_drain(&q_full[1], 0);
         for (int i = (kc > NS ? kc - NS : 0); i < kc; ++i) mbar_wait_drain(&k_full[i % NS], (i / NS) & 1);
         for (int i = (vc > NS ? vc - NS : 0); i < vc; ++i) mbar_wait_drain(&v_full[i % NS], (i / NS) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_addr(sQ);
       const uint32_t k_base = smem_addr(sK);
       const uint32_t v_base = smem_addr(sV);
-      const uint32_t p_base = smem_addr(sP);
-      int kc = 0, vc = 0, sc = 0;
-      bool ok = mbar_wait(q_full, 0, wc);
-      // O += P_t V_t once the softmax warps have written P_t.
-      auto issue_pv = [&](int t) -> bool {
-        if (!mbar_wait(p_full, t & 1, wc)) return false;
-        const int vs = vc % NS;
-        if (!mbar_wait(&v_full[vs], (vc / NS) & 1, wc)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(p_base + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(v_base + vs * Lay::KV_BYTES + kk * 2048, BN * 128, 1024);
-          umma_bf16_ss(tmem + Lay::TMEM_O, a, b, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+      int kc = 0, vc = 0;
+      int pc[2] = {0, 0};  // P_t consumed (pass 1)
+      int fc[2] = {0, 0};  // S_t uses in pass 2
+      bool ok = true;
+      bool q_ready[2] = {false, false};
+      // S_t = Q_t K^T into S_t's TMEM columns, from K stage ks.
+      auto issue_s = [&](int t, int ks) -> bool {
+        if (!q_ready[t]) {
+          if (!mbar_wait(&q_full[t], 0, wc)) return false;
+          q_ready[t] = true;
         }
-        umma_commit(pv_done);
-        umma_commit(&v_empty[vs]);
-        ++vc;
+        tc_fence_after();
+        const uint32_t qb = q_base + t * Lay::Q_BYTES;
+        const uint32_t d_tmem = tmem + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(qb + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sdesc_sw128(k_base + ks * Lay::KV_BYTES + (kk >> 2) * (BN * 128) +
+                                             (kk & 3) * 32, 16, 1024);
+          umma_bf16_ss(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[t]);
         return true;
       };
-      constexpr int n_pass = kDense ? 2 : 1;
-      for (int pass = 0; pass < n_pass && ok; ++pass) {
-        for (int it = 0; it < n_iter; ++it) {
-          const int ks = kc % NS;
-          if (!mbar_wait(&k_full[ks], (kc / NS) & 1, wc)) { ok = false; break; }
-          const int sb = sc & 1;
-          if (!mbar_wait(&s_free[sb], ((sc >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-          tc_fence_after();
+      auto wait_k = [&](int& ks) -> bool {
+        ks = kc % NS;
+        return mbar_wait(&k_full[ks], (kc / NS) & 1, wc);
+      };
+      auto release_k = [&](int ks) {
+        umma_commit(&k_empty[ks]);
+        ++kc;
+      };
+      // O_t += P_t V (P_t from TMEM), from V stage vs.
+      auto issue_pv = [&](int t, int vs) -> bool {
+        if (!mbar_wait(&p_full[t], pc[t] & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
+        const uint32_t d_tmem = tmem + (t ? Lay::TMEM_O1 : Lay::TMEM_O0);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            const uint32_t koff = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-            const uint64_t a = sdesc_sw128(q_base + off, 16, 1024);
-            const uint64_t b = sdesc_sw128(k_base + ks * Lay::KV_BYTES + koff, 16, 1024);
-            umma_bf16_ss(tmem + sb * BN, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t b = sdesc_sw128(v_base + vs * Lay::KV_BYTES + kk * 2048, BN * 128, 1024);
+          umma_bf16_ts(d_tmem, a_tmem + kk * 8, b, IDESC_PV, (pc[t] > 0 || kk > 0) ? 1u : 0u);
+        }
+        ++pc[t];
+        return true;
+      };
+      auto wait_v = [&](int& vs) -> bool {
+        vs = vc % NS;
+        return mbar_wait(&v_full[vs], (vc / NS) & 1, wc);
+      };
+      auto release_v = [&](int vs) {
+        umma_commit(&v_empty[vs]);
+        ++vc;
+      };
+
+      if constexpr (kDense) {
+        const int n = p.n_kv;
+        int ks, vs;
+        // ---- pass 1
+        ok = wait_k(ks) && issue_s(0, ks) && issue_s(1, ks);
+        if (ok) release_k(ks);
+        for (int j = 0; ok && j < n; ++j) {
+          if (!(ok = wait_v(vs))) break;
+          if (!(ok = issue_pv(0, vs))) break;
+          int ks2 = -1;
+          if (j + 1 < n) {
+            if (!(ok = wait_k(ks2) && issue_s(0, ks2))) break;
+          } else {
+            umma_commit(&o_full[0]);
           }
-          umma_commit(&s_full[sb]);
-          umma_commit(&k_empty[ks]);
-          ++kc;
-          ++sc;
-          if (pass == 0 && it > 0) {
-            if (!issue_pv(it - 1)) { ok = false; break; }
+          if (!(ok = issue_pv(1, vs))) break;
+          release_v(vs);
+          if (j + 1 < n) {
+            if (!(ok = issue_s(1, ks2))) break;
+            release_k(ks2);
+          } else {
+            umma_commit(&o_full[1]);
           }
         }
-        if (ok && pass == 0 && n_iter > 0) ok = issue_pv(n_iter - 1);
+        // ---- pass 2: S only; S_t is free again once softmax t has read it
+        for (int j = 0; ok && j < n; ++j) {
+          if (!(ok = wait_k(ks))) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (ok && fc[t] > 0) ok = mbar_wait(&s_free[t], (fc[t] - 1) & 1, wc);
+            if (ok) ok = issue_s(t, ks);
+            ++fc[t];
+          }
+          if (!ok) break;
+          release_k(ks);
+        }
+      } else {
+        int ks, vs;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (ok && n_it[t] > 0) {
+            ok = wait_k(ks) && issue_s(t, ks);
+            if (ok) release_k(ks);
+          }
+        }
+        const int n_max = max(n_it[0], n_it[1]);
+        for (int j = 0; ok && j < n_max; ++j) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || j >= n_it[t]) continue;
+            ok = wait_v(vs) && issue_pv(t, vs);
+            if (!ok) break;
+            release_v(vs);
+            if (j + 1 < n_it[t]) {
+              ok = wait_k(ks) && issue_s(t, ks);
+              if (!ok) break;
+              release_k(ks);
+            } else {
+              umma_commit(&o_full[t]);
+            }
+          }
+        }
       }
       if (!ok) {
         // Drain: let every MMA issued so far finish before TMEM is freed.
@@ -254,13 +369,20 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait_drain(drain_bar, 0);
       }
     }
+  }
   } else {
+    reg_alloc<kSoftmaxRegs>();
     // ================================================================ softmax warps
-    const int r = threadIdx.x;             // row within the tile, TMEM lane
-    const int row = qt * BM + r;           // token row within the head
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const int t = warp >> 2;               // query tile of this warpgroup
+    const int wl = warp & 3;               // warp within the warpgroup
+    const int r = wl * 32 + lane;          // row within the tile, TMEM lane
+    const int row = qt[t] * BM + r;        // token row within the head
+    const uint32_t lane_base = uint32_t(wl * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
+    const uint32_t o_col = tmem + lane_base + (t ? Lay::TMEM_O1 : Lay::TMEM_O0);
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
+    const int n = n_it[t];
     float m_used = NEG_INF;  // running max in log2 units (lazily raised)
     // Running sum of exp2(s*sl2 - m_used) in fp32, which gives lse. A row
     // sums ~10^5 terms, so each tile's terms are summed first and the tile
@@ -269,30 +391,25 @@ __global__ void __launch_bounds__(192, 1)
     float l = 0.f, l_c = 0.f;
     float lb = 0.f;          // the same sum over the bf16-rounded weights P.V uses:
                              // O = acc / lb is an exact convex combination of V rows
-    int sc = 0;
+    int sc = 0;              // S_t completions seen
     bool ok = true;
-    uint8_t* prow = sP + r * 128;
-    const int sw = r & 7;
 
-    for (int it = 0; it < n_iter; ++it) {
-      const int sb = sc & 1;
-      if (!mbar_wait(&s_full[sb], (sc >> 1) & 1, wc)) { ok = false; break; }
+    for (int j = 0; j < n; ++j) {
+      if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
+      ++sc;
       tc_fence_after();
       float s[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c)
-        tmem_ld32(tmem + lane_base + sb * BN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+        tmem_ld32(s_col + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
-      ++sc;
 
       int key0;
       bool row_on = true;
       if constexpr (kDense) {
-        key0 = it * BN;
+        key0 = j * BN;
       } else {
-        const int e = p.tile_entry[e_begin + it];
+        const int e = p.tile_entry[e_begin[t] + j];
         key0 = (e & 0xFFFF) * BN;
         row_on = ((e >> 16) >> (r / p.block)) & 1;
       }
@@ -309,85 +426,78 @@ __global__ void __launch_bounds__(192, 1)
       for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
       const float mx2 = mx * sl2;
 
-      if (it > 0) {
-        if (!mbar_wait(pv_done, (it - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-      }
       // Lazy rescale: raise the reference max only when it grows by > 8
       // (a factor 256), so exp2 values stay <= 256 and O is rarely touched.
+      // S_t(j) completing implies PV_t(j-1) completed, so O_t is at rest.
       float alpha = 1.f;
       if (mx2 > m_used + 8.f) {
         if (m_used != NEG_INF) alpha = ex2_approx(m_used - mx2);
         m_used = mx2;
       }
-      if (__any_sync(0xffffffffu, alpha != 1.f) && it > 0) {
+      if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
         l *= alpha;
         l_c *= alpha;
         lb *= alpha;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
-          tmem_ld32(tmem + lane_base + Lay::TMEM_O + c * 32, o);
+          tmem_ld32(o_col + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tmem + lane_base + Lay::TMEM_O + c * 32, o);
+          tmem_st32(o_col + c * 32, o);
         }
-        tmem_st_wait();
       }
       const float msub = (m_used == NEG_INF) ? 0.f : m_used;
       float tsum = 0.f, tsum_b = 0.f;
 #pragma unroll
-      for (int g = 0; g < BN / 8; ++g) {
-        float e[8];
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) e[j] = ex2_approx(fmaf(s[g * 8 + j], sl2, -msub));
-        tsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-        uint4 pk;
-        pk.x = pack_bf16x2(e[0], e[1]);
-        pk.y = pack_bf16x2(e[2], e[3]);
-        pk.z = pack_bf16x2(e[4], e[5]);
-        pk.w = pack_bf16x2(e[6], e[7]);
-        tsum_b += (bf16x2_sum(pk.x) + bf16x2_sum(pk.y)) + (bf16x2_sum(pk.z) + bf16x2_sum(pk.w));
-        const int slab = g >> 3, ch = g & 7;
-        *reinterpret_cast<uint4*>(prow + slab * (BM * 128) + ((ch ^ sw) << 4)) = pk;
+        for (int g = 0; g < 4; ++g) {
+          float e[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) e[i] = ex2_approx(fmaf(s[c * 32 + g * 8 + i], sl2, -msub));
+          tsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) pk[g * 4 + i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+          tsum_b += (bf16x2_sum(pk[g * 4]) + bf16x2_sum(pk[g * 4 + 1])) +
+                    (bf16x2_sum(pk[g * 4 + 2]) + bf16x2_sum(pk[g * 4 + 3]));
+        }
+        tmem_st16(s_col + c * 16, pk);
       }
       {  // Kahan: l += tsum
         const float y = tsum - l_c;
-        const float t = l + y;
-        l_c = (t - l) - y;
-        l = t;
+        const float tt = l + y;
+        l_c = (tt - l) - y;
+        l = tt;
       }
       lb += tsum_b;
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[t]);
     }
 
-    // ---- epilogue of pass 1: O = acc / l, lse
-    const bool row_in = row < p.L_pad;
-    const bool row_valid = row < p.L;
+    // ---- epilogue of pass 1: O = acc / lb, lse
+    const bool row_in = row < p.L_pad && n > 0;
+    const bool row_valid = row < p.L && n > 0;
     const float lse2 = (l > 0.f) ? m_used + log2f(l) : __int_as_float(0x7f800000);
-    if (ok && n_iter > 0) {
-      if (!mbar_wait(pv_done, (n_iter - 1) & 1, wc)) ok = false;
+    if (ok && n > 0) {
+      if (!mbar_wait(&o_full[t], 0, wc)) ok = false;
       tc_fence_after();
     }
-    if (ok) {
+    if (ok && n > 0) {
       const float inv_l = (row_valid && lb > 0.f) ? 1.f / lb : 0.f;
-      const size_t obase = (size_t(bh) * p.L_pad + row) * D;
+      const size_t obase = (size_t(bh[t]) * p.L_pad + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        if (n_iter > 0) {
-          tmem_ld32(tmem + lane_base + Lay::TMEM_O + c * 32, o);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
-        }
+        tmem_ld32(o_col + c * 32, o);
+        tmem_ld_wait();
         if (row_in) {
           if constexpr (kOutBf16) {
-            uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.o) + obase + c * 32);
+            uint32_t* dst =
+                reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.o) + obase + c * 32);
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint4 w;
@@ -407,7 +517,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       if (row_in && p.lse != nullptr)
-        p.lse[size_t(bh) * p.L_pad + row] =
+        p.lse[size_t(bh[t]) * p.L_pad + row] =
             (row_valid && l > 0.f) ? lse2 * 0.69314718055994531f : NEG_INF;
     }
 
@@ -417,35 +527,37 @@ __global__ void __launch_bounds__(192, 1)
       const int blk = p.block;
       const int nkb = BN / blk;          // key blocks per key tile (blk <= BN)
       const int q_local = r / blk;       // query block within the tile
-      const int I = qt * (BM / blk) + q_local;
+      const int I = qt[t] * (BM / blk) + q_local;
       const int n_valid_I = min(blk, p.L - I * blk);
       const float inv_cnt = (n_valid_I > 0) ? 1.f / float(n_valid_I) : 0.f;
       const float lsub = row_valid ? lse2 : __int_as_float(0x7f800000);
       const int wpb = blk / 32;          // warps per query block (1, 2 or 4)
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const int sb = sc & 1;
-        if (!mbar_wait(&s_full[sb], (sc >> 1) & 1, wc)) { ok = false; break; }
+      float* red_t = red + t * 32;
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
+        ++sc;
         tc_fence_after();
         float s[BN];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c)
-          tmem_ld32(tmem + lane_base + sb * BN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+          tmem_ld32(s_col + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&s_free[sb]);
-        ++sc;
+        mbar_arrive(&s_free[t]);
 
-        const int key0 = it * BN;
+        const int key0 = j * BN;
         float part[NKB_MAX];
 #pragma unroll
-        for (int kb = 0; kb < NKB_MAX; ++kb) part[kb] = 0.f;
+        for (int g = 0; g < NKB_MAX; ++g) {
+          float acc = 0.f;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          // Padded query rows and padded keys contribute nothing (and may
-          // hold any finite or non-finite score).
-          const float e =
-              (row_valid && key0 + c < p.L) ? ex2_approx(fmaf(s[c], sl2, -lsub)) : 0.f;
-          part[c / 32] += e;   // 32-column groups; merged into key blocks below
+          for (int c = 0; c < 32; ++c) {
+            // Padded query rows and padded keys contribute nothing (and may
+            // hold any finite or non-finite score).
+            const int col = g * 32 + c;
+            acc += (row_valid && key0 + col < p.L) ? ex2_approx(fmaf(s[col], sl2, -lsub)) : 0.f;
+          }
+          part[g] = acc;
         }
         // Merge 32-column groups into key blocks of size blk.
         float kbsum[NKB_MAX];
@@ -465,22 +577,22 @@ __global__ void __launch_bounds__(192, 1)
           if (lane == 0 && I < p.n_blocks) {
             for (int kb = 0; kb < nkb; ++kb)
               if (J0 + kb < p.n_blocks)
-                p.mass[(size_t(bh) * p.n_blocks + I) * p.n_blocks + J0 + kb] = kbsum[kb] * inv_cnt;
+                p.mass[(size_t(bh[t]) * p.n_blocks + I) * p.n_blocks + J0 + kb] = kbsum[kb] * inv_cnt;
           }
         } else {
-          float* rb = red + (it & 1) * 16;
+          float* rb = red_t + (j & 1) * 16;
           if (lane == 0) {
 #pragma unroll
-            for (int kb = 0; kb < NKB_MAX; ++kb) rb[warp * 4 + kb] = kbsum[kb];
+            for (int kb = 0; kb < NKB_MAX; ++kb) rb[wl * 4 + kb] = kbsum[kb];
           }
-          mbar_arrive(&red_bar[it & 1]);
-          if (!mbar_wait(&red_bar[it & 1], (it >> 1) & 1, wc)) { ok = false; break; }
-          if (lane == 0 && (warp % wpb) == 0 && I < p.n_blocks) {
+          mbar_arrive(&red_bar[2 * t + (j & 1)]);
+          if (!mbar_wait(&red_bar[2 * t + (j & 1)], (j >> 1) & 1, wc)) { ok = false; break; }
+          if (lane == 0 && (wl % wpb) == 0 && I < p.n_blocks) {
             for (int kb = 0; kb < nkb; ++kb) {
-              float t = 0.f;
-              for (int w = warp; w < warp + wpb; ++w) t += rb[w * 4 + kb];
+              float tot = 0.f;
+              for (int w = wl; w < wl + wpb; ++w) tot += rb[w * 4 + kb];
               if (J0 + kb < p.n_blocks)
-                p.mass[(size_t(bh) * p.n_blocks + I) * p.n_blocks + J0 + kb] = t * inv_cnt;
+                p.mass[(size_t(bh[t]) * p.n_blocks + I) * p.n_blocks + J0 + kb] = tot * inv_cnt;
             }
           }
         }
@@ -490,7 +602,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, Lay::TMEM_COLS);
