@@ -44,18 +44,19 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int L_pad, int d, int 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, int NS, bool kDense, bool kOutBf16>
+template <int D, int BN, int NS, bool kDense, bool kOutBf16, int BLK>
 cudaError_t run(const void* q, const void* k, const void* v, int BH, const AttnParams& p,
                 dim3 grid, cudaStream_t stream) {
   using Lay = AttnLayout<D, BN, NS>;
-  auto kern = attn_kernel<D, BN, NS, kDense, kOutBf16>;
+  auto kern = attn_kernel<D, BN, NS, kDense, kOutBf16, BLK>;
   // Cheap, and per device: set on every launch.
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM_ALLOC);
   if (err != cudaSuccess) return err;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, BH, p.L_pad, D, 128) || !make_map(&tk, k, BH, p.L_pad, D, BN) ||
-      !make_map(&tv, v, BH, p.L_pad, D, BN))
+  constexpr int box = kDense ? BN : BLK;
+  if (!make_map(&tq, q, BH, p.L_pad, D, 128) || !make_map(&tk, k, BH, p.L_pad, D, box) ||
+      !make_map(&tv, v, BH, p.L_pad, D, box))
     return cudaErrorInvalidValue;
   kern<<<grid, kAttnThreads, Lay::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
@@ -101,12 +102,18 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, in
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
   const dim3 grid((p.n_qt + 1) / 2, BH);  // two query tiles per CTA
-  if (d == 128) {
-    return out_bf16 ? run<128, 128, 2, true, true>(q, k, v, BH, p, grid, stream)
-                    : run<128, 128, 2, true, false>(q, k, v, BH, p, grid, stream);
-  }
-  return out_bf16 ? run<64, 128, 4, true, true>(q, k, v, BH, p, grid, stream)
-                  : run<64, 128, 4, true, false>(q, k, v, BH, p, grid, stream);
+#define LOSA_DENSE_CASE(D_, NS_, BLK_)                                                     \
+  if (d == D_ && block == BLK_)                                                           \
+    return out_bf16 ? run<D_, 128, NS_, true, true, BLK_>(q, k, v, BH, p, grid, stream)  \
+                    : run<D_, 128, NS_, true, false, BLK_>(q, k, v, BH, p, grid, stream);
+  LOSA_DENSE_CASE(128, 2, 128)
+  LOSA_DENSE_CASE(128, 2, 64)
+  LOSA_DENSE_CASE(128, 2, 32)
+  LOSA_DENSE_CASE(64, 4, 128)
+  LOSA_DENSE_CASE(64, 4, 64)
+  LOSA_DENSE_CASE(64, 4, 32)
+#undef LOSA_DENSE_CASE
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, int L,
@@ -132,16 +139,16 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, in
   p.n_tiles = int(pat->n_tiles);
   const dim3 grid(unsigned((pat->n_tiles + 1) / 2));  // two tiles per CTA
   if (pat->n_tiles == 0) return cudaSuccess;
-#define LOSA_SPARSE_CASE(D_, BN_, NS_)                                                    \
-  if (d == D_ && pat->block == BN_)                                                      \
-    return out_bf16 ? run<D_, BN_, NS_, false, true>(q, k, v, BH, p, grid, stream)      \
-                    : run<D_, BN_, NS_, false, false>(q, k, v, BH, p, grid, stream);
-  LOSA_SPARSE_CASE(128, 128, 2)
-  LOSA_SPARSE_CASE(128, 64, 4)
-  LOSA_SPARSE_CASE(128, 32, 8)
-  LOSA_SPARSE_CASE(64, 128, 4)
-  LOSA_SPARSE_CASE(64, 64, 8)
-  LOSA_SPARSE_CASE(64, 32, 8)
+#define LOSA_SPARSE_CASE(D_, NS_, BLK_)                                                     \
+  if (d == D_ && pat->block == BLK_)                                                       \
+    return out_bf16 ? run<D_, 128, NS_, false, true, BLK_>(q, k, v, BH, p, grid, stream)  \
+                    : run<D_, 128, NS_, false, false, BLK_>(q, k, v, BH, p, grid, stream);
+  LOSA_SPARSE_CASE(128, 2, 128)
+  LOSA_SPARSE_CASE(128, 2, 64)
+  LOSA_SPARSE_CASE(128, 2, 32)
+  LOSA_SPARSE_CASE(64, 4, 128)
+  LOSA_SPARSE_CASE(64, 4, 64)
+  LOSA_SPARSE_CASE(64, 4, 32)
 #undef LOSA_SPARSE_CASE
   return cudaErrorInvalidValue;
 }

@@ -83,18 +83,26 @@ struct AttnLayout {
 
 constexpr int kAttnThreads = 384;
 constexpr int kAttnLaunchRegs = 168;   // checked against ptxas at build time
-constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kAttnThreads * kAttnLaunchRegs,
               "register split must use exactly the launch allocation");
 
-template <int D, int BN, int NS, bool kDense, bool kOutBf16>
+// BLK: the LoSA block size b (compile time, so that every per-block array
+// stays in registers). Dense: key tiles of BN = 128 rows, one TMA box each;
+// the mass pass sums over b x b blocks. Sparse: each 128-key iteration packs
+// EPI = BN / b consecutive entries of the tile's list into one K/V stage
+// (one b-row box each, stacked), so the tensor core always runs N = 128.
+template <int D, int BN, int NS, bool kDense, bool kOutBf16, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using Lay = AttnLayout<D, BN, NS>;
   constexpr int BM = Lay::BM;
   constexpr int N_SLABS = D / 64;
+  constexpr int BOX = kDense ? BN : BLK;  // key rows per TMA box
+  constexpr int EPI = BN / BOX;           // boxes (list entries) per key stage
+  static_assert(BN % BLK == 0 && BLK % 32 == 0, "block size");
   constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
 
@@ -124,7 +132,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work items: per tile t, its head, query tile and key list
-  int bh[2], qt[2], e_begin[2] = {0, 0}, n_it[2];
+  int bh[2], qt[2], e_begin[2] = {0, 0}, n_ent[2] = {0, 0}, n_it[2];
   if constexpr (kDense) {
     bh[0] = bh[1] = blockIdx.y;
     qt[0] = 2 * blockIdx.x;
@@ -139,7 +147,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bh[t] = tile / p.n_qt;
         qt[t] = tile - bh[t] * p.n_qt;
         e_begin[t] = p.tile_ptr[tile];
-        n_it[t] = p.tile_ptr[tile + 1] - e_begin[t];
+        n_ent[t] = p.tile_ptr[tile + 1] - e_begin[t];
+        n_it[t] = (n_ent[t] + EPI - 1) / EPI;
       } else {
         bh[t] = 0;
         qt[t] = 0;
@@ -193,39 +202,55 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       int kc = 0, vc = 0;
       bool ok = true;
-      auto load_k = [&](int key_row, int head) -> bool {
+      // One stage = BN keys = EPI boxes of BLK rows, stacked in each slab.
+      auto load_k = [&](const int (&key_row)[EPI], int head) -> bool {
         const int ks = kc % NS;
         if (!mbar_wait(&k_empty[ks], ((kc / NS) & 1) ^ 1, wc)) return false;
         mbar_arrive_expect_tx(&k_full[ks], Lay::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < N_SLABS; ++s)
-          tma_load_3d(sK + ks * Lay::KV_BYTES + s * (BN * 128), &tm_k, &k_full[ks], s * 64,
-                      key_row, head);
+#pragma unroll
+          for (int e = 0; e < EPI; ++e)
+            tma_load_3d(sK + ks * Lay::KV_BYTES + s * (BN * 128) + e * (BOX * 128), &tm_k,
+                        &k_full[ks], s * 64, key_row[e], head);
         ++kc;
         return true;
       };
-      auto load_v = [&](int key_row, int head) -> bool {
+      auto load_v = [&](const int (&key_row)[EPI], int head) -> bool {
         const int vs = vc % NS;
         if (!mbar_wait(&v_empty[vs], ((vc / NS) & 1) ^ 1, wc)) return false;
         mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < N_SLABS; ++s)
-          tma_load_3d(sV + vs * Lay::KV_BYTES + s * (BN * 128), &tm_v, &v_full[vs], s * 64,
-                      key_row, head);
+#pragma unroll
+          for (int e = 0; e < EPI; ++e)
+            tma_load_3d(sV + vs * Lay::KV_BYTES + s * (BN * 128) + e * (BOX * 128), &tm_v,
+                        &v_full[vs], s * 64, key_row[e], head);
         ++vc;
         return true;
       };
       if constexpr (kDense) {
-        for (int j = 0; ok && j < p.n_kv; ++j) ok = load_k(j * BN, bh[0]) && load_v(j * BN, bh[0]);
-        for (int j = 0; ok && j < p.n_kv; ++j) ok = load_k(j * BN, bh[0]);
+        for (int j = 0; ok && j < p.n_kv; ++j) {
+          const int rows[EPI] = {j * BN};
+          ok = load_k(rows, bh[0]) && load_v(rows, bh[0]);
+        }
+        for (int j = 0; ok && j < p.n_kv; ++j) {
+          const int rows[EPI] = {j * BN};
+          ok = load_k(rows, bh[0]);
+        }
       } else {
         const int n_max = max(n_it[0], n_it[1]);
         for (int j = 0; ok && j < n_max; ++j) {
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (ok && j < n_it[t]) {
-              const int row = (p.tile_entry[e_begin[t] + j] & 0xFFFF) * BN;
-              ok = load_k(row, bh[t]) && load_v(row, bh[t]);
+              // Slots past the end of the list repeat its last entry (valid,
+              // finite data); the softmax masks those columns.
+              int rows[EPI];
+#pragma unroll
+              for (int e = 0; e < EPI; ++e)
+                rows[e] = (p.tile_entry[e_begin[t] + min(j * EPI + e, n_ent[t] - 1)] & 0xFFFF) * BLK;
+              ok = load_k(rows, bh[t]) && load_v(rows, bh[t]);
             }
           }
         }
@@ -382,7 +407,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t o_col = tmem + lane_base + (t ? Lay::TMEM_O1 : Lay::TMEM_O0);
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    const int n = n_it[t];
+    const int n_iter = n_it[t];
+    const int n = kDense ? n_iter : n_ent[t];  // list entries (sparse)
     float m_used = NEG_INF;  // running max in log2 units (lazily raised)
     // Running sum of exp2(s*sl2 - m_used) in fp32, which gives lse. A row
     // sums ~10^5 terms, so each tile's terms are summed first and the tile
@@ -394,7 +420,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int sc = 0;              // S_t completions seen
     bool ok = true;
 
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < n_iter; ++j) {
+      // The list entries of this iteration: fetched before waiting for S so
+      // the global-load latency hides behind the wait. Past the end: off.
+      int ent[EPI];
+      if constexpr (!kDense) {
+#pragma unroll
+        for (int e = 0; e < EPI; ++e) {
+          const int idx = j * EPI + e;
+          ent[e] = (idx < n) ? __ldg(p.tile_entry + e_begin[t] + idx) : 0;
+        }
+      }
       if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
       ++sc;
       tc_fence_after();
@@ -404,26 +440,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32(s_col + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
       tmem_ld_wait();
 
-      int key0;
-      bool row_on = true;
+      // Key padding (only in the head's last key block) masks columns of S;
+      // a sparse entry whose query block does not keep it is masked as a
+      // whole through its exponent offset below, leaving S untouched.
+      bool on[EPI];
       if constexpr (kDense) {
-        key0 = j * BN;
+        on[0] = true;
+        const int key0 = j * BN;
+        if (key0 + BN > p.L) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (key0 + c >= p.L) s[c] = NEG_INF;
+        }
       } else {
-        const int e = p.tile_entry[e_begin[t] + j];
-        key0 = (e & 0xFFFF) * BN;
-        row_on = ((e >> 16) >> (r / p.block)) & 1;
+        // A warp's 32 rows lie in one query block (BLK >= 32): warp-uniform.
+        const int qb = r / BLK;
+#pragma unroll
+        for (int e = 0; e < EPI; ++e) {
+          const int key0 = (ent[e] & 0xFFFF) * BLK;
+          on[e] = ((ent[e] >> 16) >> qb) & 1;
+          if (key0 + BLK > p.L) {
+#pragma unroll
+            for (int c = 0; c < BLK; ++c)
+              if (key0 + c >= p.L) s[e * BLK + c] = NEG_INF;
+          }
+        }
       }
-      if (!row_on) {
+      // Row max over the kept entries: per entry a tree over 8 independent
+      // partial maxima (a serial chain would expose the FMNMX latency once
+      // per column), then combined under the entry flags.
+      float mx = NEG_INF;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = NEG_INF;
-      } else if (key0 + BN > p.L) {
+      for (int e = 0; e < EPI; ++e) {
+        float pm[8];
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (key0 + c >= p.L) s[c] = NEG_INF;
+        for (int i = 0; i < 8; ++i) pm[i] = s[e * BOX + i];
+#pragma unroll
+        for (int c = 8; c < BOX; ++c) pm[c & 7] = fmaxf(pm[c & 7], s[e * BOX + c]);
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) pm[i] = fmaxf(pm[i], pm[i + w]);
+        mx = on[e] ? fmaxf(mx, pm[0]) : mx;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
       const float mx2 = mx * sl2;
 
       // Lazy rescale: raise the reference max only when it grows by > 8
@@ -449,6 +508,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       const float msub = (m_used == NEG_INF) ? 0.f : m_used;
+      // Exponent offset per entry: -msub, or -inf for an entry this row's
+      // query block does not keep (S is finite there, so exp2 gives 0).
+      float nsub[EPI];
+#pragma unroll
+      for (int e = 0; e < EPI; ++e) nsub[e] = on[e] ? -msub : NEG_INF;
       float tsum = 0.f, tsum_b = 0.f;
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
@@ -457,7 +521,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int g = 0; g < 4; ++g) {
           float e[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) e[i] = ex2_approx(fmaf(s[c * 32 + g * 8 + i], sl2, -msub));
+          for (int i = 0; i < 8; ++i)
+            e[i] = ex2_approx(fmaf(s[c * 32 + g * 8 + i], sl2, nsub[(c * 32 + g * 8) / BOX]));
           tsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
 #pragma unroll
           for (int i = 0; i < 4; ++i) pk[g * 4 + i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
@@ -479,14 +544,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 
     // ---- epilogue of pass 1: O = acc / lb, lse
-    const bool row_in = row < p.L_pad && n > 0;
-    const bool row_valid = row < p.L && n > 0;
+    const bool row_in = row < p.L_pad && n_iter > 0;
+    const bool row_valid = row < p.L && n_iter > 0;
     const float lse2 = (l > 0.f) ? m_used + log2f(l) : __int_as_float(0x7f800000);
-    if (ok && n > 0) {
+    if (ok && n_iter > 0) {
       if (!mbar_wait(&o_full[t], 0, wc)) ok = false;
       tc_fence_after();
     }
-    if (ok && n > 0) {
+    if (ok && n_iter > 0) {
       const float inv_l = (row_valid && lb > 0.f) ? 1.f / lb : 0.f;
       const size_t obase = (size_t(bh[t]) * p.L_pad + row) * D;
 #pragma unroll
@@ -523,17 +588,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if constexpr (kDense) {
       // ---- pass 2: block masses from exp(s - lse)
-      constexpr int NKB_MAX = BN / 32;  // key blocks per tile for the smallest block
-      const int blk = p.block;
-      const int nkb = BN / blk;          // key blocks per key tile (blk <= BN)
-      const int q_local = r / blk;       // query block within the tile
-      const int I = qt[t] * (BM / blk) + q_local;
-      const int n_valid_I = min(blk, p.L - I * blk);
+      constexpr int NKB = BN / BLK;      // key blocks per key tile
+      constexpr int NG = BN / 32;        // 32-column groups per key tile
+      constexpr int WPB = BLK / 32;      // warps per query block (1, 2 or 4)
+      const int q_local = r / BLK;       // query block within the tile
+      const int I = qt[t] * (BM / BLK) + q_local;
+      const int n_valid_I = min(BLK, p.L - I * BLK);
       const float inv_cnt = (n_valid_I > 0) ? 1.f / float(n_valid_I) : 0.f;
       const float lsub = row_valid ? lse2 : __int_as_float(0x7f800000);
-      const int wpb = blk / 32;          // warps per query block (1, 2 or 4)
       float* red_t = red + t * 32;
-      for (int j = 0; ok && j < n; ++j) {
+      for (int j = 0; ok && j < n_iter; ++j) {
         if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
         ++sc;
         tc_fence_after();
@@ -546,53 +610,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&s_free[t]);
 
         const int key0 = j * BN;
-        float part[NKB_MAX];
+        // Padded query rows subtract +inf (their scores are finite: rows past
+        // L hold finite values by contract, rows past L_pad read as zero), so
+        // they add exact zeros. Padded keys only occur in the last key tile,
+        // which takes its own warp-uniform branch.
+        float part[NG];
+        if (key0 + BN <= p.L) {
 #pragma unroll
-        for (int g = 0; g < NKB_MAX; ++g) {
-          float acc = 0.f;
+          for (int g = 0; g < NG; ++g) {
+            // 32 columns summed as a tree of 4 independent partial sums.
+            float a[4];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            // Padded query rows and padded keys contribute nothing (and may
-            // hold any finite or non-finite score).
-            const int col = g * 32 + c;
-            acc += (row_valid && key0 + col < p.L) ? ex2_approx(fmaf(s[col], sl2, -lsub)) : 0.f;
+            for (int i = 0; i < 4; ++i) a[i] = ex2_approx(fmaf(s[g * 32 + i], sl2, -lsub));
+#pragma unroll
+            for (int c = 4; c < 32; ++c) a[c & 3] += ex2_approx(fmaf(s[g * 32 + c], sl2, -lsub));
+            part[g] = (a[0] + a[1]) + (a[2] + a[3]);
           }
-          part[g] = acc;
+        } else {
+          const int lim = p.L - key0;
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              a[c & 3] += (g * 32 + c < lim) ? ex2_approx(fmaf(s[g * 32 + c], sl2, -lsub)) : 0.f;
+            part[g] = (a[0] + a[1]) + (a[2] + a[3]);
+          }
         }
-        // Merge 32-column groups into key blocks of size blk.
-        float kbsum[NKB_MAX];
+        // Merge 32-column groups into key blocks of BLK columns.
+        float kbsum[NKB];
 #pragma unroll
-        for (int kb = 0; kb < NKB_MAX; ++kb) kbsum[kb] = 0.f;
+        for (int kb = 0; kb < NKB; ++kb) kbsum[kb] = 0.f;
 #pragma unroll
-        for (int g = 0; g < NKB_MAX; ++g) kbsum[(g * 32) / blk] += part[g];
+        for (int g = 0; g < NG; ++g) kbsum[(g * 32) / BLK] += part[g];
         // Sum over the rows of this warp.
 #pragma unroll
-        for (int kb = 0; kb < NKB_MAX; ++kb) {
+        for (int kb = 0; kb < NKB; ++kb) {
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1)
             kbsum[kb] += __shfl_xor_sync(0xffffffffu, kbsum[kb], off);
         }
-        const int J0 = key0 / blk;
-        if (wpb == 1) {
+        const int J0 = key0 / BLK;
+        float* mrow = p.mass + (size_t(bh[t]) * p.n_blocks + I) * p.n_blocks;
+        if constexpr (WPB == 1) {
           if (lane == 0 && I < p.n_blocks) {
-            for (int kb = 0; kb < nkb; ++kb)
-              if (J0 + kb < p.n_blocks)
-                p.mass[(size_t(bh[t]) * p.n_blocks + I) * p.n_blocks + J0 + kb] = kbsum[kb] * inv_cnt;
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb)
+              if (J0 + kb < p.n_blocks) mrow[J0 + kb] = kbsum[kb] * inv_cnt;
           }
         } else {
           float* rb = red_t + (j & 1) * 16;
           if (lane == 0) {
 #pragma unroll
-            for (int kb = 0; kb < NKB_MAX; ++kb) rb[wl * 4 + kb] = kbsum[kb];
+            for (int kb = 0; kb < NKB; ++kb) rb[wl * 4 + kb] = kbsum[kb];
           }
           mbar_arrive(&red_bar[2 * t + (j & 1)]);
           if (!mbar_wait(&red_bar[2 * t + (j & 1)], (j >> 1) & 1, wc)) { ok = false; break; }
-          if (lane == 0 && (wl % wpb) == 0 && I < p.n_blocks) {
-            for (int kb = 0; kb < nkb; ++kb) {
+          if (lane == 0 && (wl % WPB) == 0 && I < p.n_blocks) {
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) {
               float tot = 0.f;
-              for (int w = wl; w < wl + wpb; ++w) tot += rb[w * 4 + kb];
-              if (J0 + kb < p.n_blocks)
-                p.mass[(size_t(bh[t]) * p.n_blocks + I) * p.n_blocks + J0 + kb] = tot * inv_cnt;
+#pragma unroll
+              for (int w = 0; w < WPB; ++w) tot += rb[(wl + w) * 4 + kb];
+              if (J0 + kb < p.n_blocks) mrow[J0 + kb] = tot * inv_cnt;
             }
           }
         }

@@ -272,19 +272,25 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int* __restrict__ in, 
   if (threadIdx.x == 0) out[n] = carry;
 }
 
-// Tiles ordered by entry count, largest first (longest-processing-time
-// order for the sparse kernel's block scheduler). Counting sort on
-// (n - count); order among equal counts is unspecified.
-__global__ void order_hist_kernel(const int* __restrict__ tile_count, int T, int n,
-                                  int* __restrict__ hist) {
-  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x)
-    atomicAdd(&hist[n - tile_count[t]], 1);
+// Order of the sparse kernel's work: head by head (so the CTAs resident at
+// one time gather from one head's K/V, which stays in L2), and within a
+// head by entry count, largest first (longest-processing-time order for the
+// block scheduler). Counting sort on the key head * (n + 1) + (n - count);
+// order among equal keys is unspecified.
+__device__ __forceinline__ int order_key(int t, int n_qt, int n, const int* tile_count) {
+  return (t / n_qt) * (n + 1) + (n - tile_count[t]);
 }
 
-__global__ void order_scatter_kernel(const int* __restrict__ tile_count, int T, int n,
+__global__ void order_hist_kernel(const int* __restrict__ tile_count, int T, int n_qt, int n,
+                                  int* __restrict__ hist) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x)
+    atomicAdd(&hist[order_key(t, n_qt, n, tile_count)], 1);
+}
+
+__global__ void order_scatter_kernel(const int* __restrict__ tile_count, int T, int n_qt, int n,
                                      int* __restrict__ cursor, int* __restrict__ order) {
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x)
-    order[atomicAdd(&cursor[n - tile_count[t]], 1)] = t;
+    order[atomicAdd(&cursor[order_key(t, n_qt, n, tile_count)], 1)] = t;
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -324,9 +330,10 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
   const size_t s_cut = 0;
   const size_t s_cnt = s_cut + align256(R * 8);
   const size_t s_tcnt = s_cnt + align256(R * 4);
+  const int64_t n_keys = int64_t(BH) * (n + 1);  // order keys: head x (n + 1)
   const size_t s_hist = s_tcnt + align256(T * 4);
-  const size_t s_cur = s_hist + align256((n + 1) * 4);
-  const size_t scratch_bytes = s_cur + align256((n + 2) * 4);
+  const size_t s_cur = s_hist + align256(n_keys * 4);
+  const size_t scratch_bytes = s_cur + align256((n_keys + 1) * 4);
 
   char* fixed = static_cast<char*>(pool_alloc(fixed_bytes, stream));
   char* scratch = static_cast<char*>(pool_alloc(scratch_bytes, stream));
@@ -356,11 +363,11 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
   tile_count_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(mass, cut, n, qpt, n_qt, tcnt);
   scan_kernel<<<1, 1024, 0, stream>>>(cnt, int(R), p->row_ptr);
   scan_kernel<<<1, 1024, 0, stream>>>(tcnt, int(T), p->tile_ptr);
-  cudaMemsetAsync(hist, 0, (n + 1) * sizeof(int), stream);
+  cudaMemsetAsync(hist, 0, n_keys * sizeof(int), stream);
   const int og = int(std::min<int64_t>((T + 255) / 256, 1024));
-  order_hist_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n, hist);
-  scan_kernel<<<1, 1024, 0, stream>>>(hist, n + 1, cursor);
-  order_scatter_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n, cursor, p->tile_order);
+  order_hist_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n_qt, n, hist);
+  scan_kernel<<<1, 1024, 0, stream>>>(hist, int(n_keys), cursor);
+  order_scatter_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n_qt, n, cursor, p->tile_order);
   if (cudaGetLastError() != cudaSuccess) return fail(LOSA_ERR_CUDA);
 
   // The one host synchronisation: CSR sizes and the mass check.

@@ -64,7 +64,8 @@ def assert_lse_close(lse_gpu, lse_ref, L):
 
 def check_tiles(ex, pat, n):
     """The sparse kernel's work list is the per-tile union of the rows'
-    kept sets, with correct masks, ordered by entry count (largest first)."""
+    kept sets, with correct masks, ordered head by head and, within a head,
+    by entry count (largest first)."""
     row_ptr = ex["row_ptr"].numpy()
     col_idx = ex["col_idx"].numpy()
     tile_ptr = ex["tile_ptr"].numpy()
@@ -74,7 +75,10 @@ def check_tiles(ex, pat, n):
     n_qt = (n * pat.block + 127) // 128
     assert sorted(order.tolist()) == list(range(pat.n_tiles))
     counts = np.diff(tile_ptr)
-    assert np.all(np.diff(counts[order]) <= 0)
+    heads = order // n_qt
+    assert np.all(np.diff(heads) >= 0)
+    same = np.diff(heads) == 0
+    assert np.all(np.diff(counts[order])[same] <= 0)
     for t in range(pat.n_tiles):
         bh, qt = divmod(t, n_qt)
         want = {}
