@@ -476,12 +476,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) pm[i] = s[e * BOX + i];
 #pragma unroll
-        for (int c = 8; c < BOX; ++c) pm[c & 7] = fmaxf(pm[c & 7], s[e * BOX + c]);
-#pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) pm[i] = fmaxf(pm[i], pm[i + w]);
-        mx = on[e] ? fmaxf(mx, pm[0]) : mx;
+        for (int c = 8; c < BOX; c += 2) pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], s[e * BOX + c], s[e * BOX + c + 1]);
+        const float m0 = fmax3(pm[0], pm[1], pm[2]);
+        const float m1 = fmax3(pm[3], pm[4], pm[5]);
+        const float m2 = fmax3(pm[6], pm[7], m0);
+        mx = on[e] ? fmax3(mx, m1, m2) : mx;
       }
       const float mx2 = mx * sl2;
 
@@ -513,24 +512,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float nsub[EPI];
 #pragma unroll
       for (int e = 0; e < EPI; ++e) nsub[e] = on[e] ? -msub : NEG_INF;
-      float tsum = 0.f, tsum_b = 0.f;
+      // exp2 of (s * sl2 + offset), two columns per packed FMA; the fp32
+      // sum (for lse) in packed adds, the bf16 sum (for O) in mixed adds.
+      const f32x2 sl2x2 = f2_make(sl2, sl2);
+      f32x2 ts2[2] = {0ull, 0ull};
+      float lbs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          float e[8];
+          const float ns = nsub[(c * 32 + g * 8) / BOX];
+          const f32x2 ns2 = f2_make(ns, ns);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            e[i] = ex2_approx(fmaf(s[c * 32 + g * 8 + i], sl2, nsub[(c * 32 + g * 8) / BOX]));
-          tsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-#pragma unroll
-          for (int i = 0; i < 4; ++i) pk[g * 4 + i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
-          tsum_b += (bf16x2_sum(pk[g * 4]) + bf16x2_sum(pk[g * 4 + 1])) +
-                    (bf16x2_sum(pk[g * 4 + 2]) + bf16x2_sum(pk[g * 4 + 3]));
+          for (int i = 0; i < 4; ++i) {
+            const int col = c * 32 + g * 8 + 2 * i;
+            float a0, a1;
+            f2_split(f2_fma(f2_make(s[col], s[col + 1]), sl2x2, ns2), a0, a1);
+            const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+            ts2[i & 1] = f2_add(ts2[i & 1], f2_make(e0, e1));
+            pk[g * 4 + i] = pack_bf16x2(e0, e1);
+            lbs[i] = add_bf16x2_to(lbs[i], pk[g * 4 + i]);
+          }
         }
         tmem_st16(s_col + c * 16, pk);
       }
+      const float tsum = f2_sum(ts2[0]) + f2_sum(ts2[1]);
+      const float tsum_b = (lbs[0] + lbs[1]) + (lbs[2] + lbs[3]);
       {  // Kahan: l += tsum
         const float y = tsum - l_c;
         const float tt = l + y;
@@ -616,15 +624,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // which takes its own warp-uniform branch.
         float part[NG];
         if (key0 + BN <= p.L) {
+          const f32x2 sl2x2 = f2_make(sl2, sl2);
+          const f32x2 nl2 = f2_make(-lsub, -lsub);
 #pragma unroll
           for (int g = 0; g < NG; ++g) {
-            // 32 columns summed as a tree of 4 independent partial sums.
-            float a[4];
+            // 32 columns: packed FMAs for the exponents, two packed partial
+            // sums (four independent fp32 lanes).
+            f32x2 acc[2] = {0ull, 0ull};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = ex2_approx(fmaf(s[g * 32 + i], sl2, -lsub));
-#pragma unroll
-            for (int c = 4; c < 32; ++c) a[c & 3] += ex2_approx(fmaf(s[g * 32 + c], sl2, -lsub));
-            part[g] = (a[0] + a[1]) + (a[2] + a[3]);
+            for (int c = 0; c < 32; c += 2) {
+              float a0, a1;
+              f2_split(f2_fma(f2_make(s[g * 32 + c], s[g * 32 + c + 1]), sl2x2, nl2), a0, a1);
+              acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_make(ex2_approx(a0), ex2_approx(a1)));
+            }
+            part[g] = f2_sum(acc[0]) + f2_sum(acc[1]);
           }
         } else {
           const int lim = p.L - key0;

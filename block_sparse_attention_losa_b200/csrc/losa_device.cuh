@@ -255,6 +255,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ---- sm_100 packed fp32 arithmetic: two fp32 lanes in one 64-bit register.
+using f32x2 = unsigned long long;
+
+__device__ __forceinline__ f32x2 f2_make(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(f32x2 r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float f2_sum(f32x2 a) {
+  float lo, hi;
+  f2_split(a, lo, hi);
+  return lo + hi;
+}
+// max of three fp32 values in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// acc + (both bf16 halves of w), each widened exactly to fp32.
+__device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "add.f32.bf16 %0, lo, %0;\n\t"
+      "add.f32.bf16 %0, hi, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(w));
+  return acc;
+}
+
 // Sum of the two bf16 values packed in a 32-bit word, in fp32 (exact
 // widening of each half).
 __device__ __forceinline__ float bf16x2_sum(uint32_t w) {
