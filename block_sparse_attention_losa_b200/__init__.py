@@ -29,7 +29,7 @@ STATUS = {0: "LOSA_OK", -1: "LOSA_ERR_ARG", -2: "LOSA_ERR_CUDA", -3: "LOSA_ERR_N
 # Every symbol include/losa.h declares.
 EXPORTS = ("losa_dense_mass", "losa_select", "losa_pattern_info", "losa_pattern_export",
            "losa_select_noalloc", "losa_sparse_attn", "losa_free", "losa_check_status",
-           "losa_strerror", "losa_version")
+           "losa_exp2_eval", "losa_strerror", "losa_version")
 NOALLOC_MAX_ROWS = 65536  # LOSA_NOALLOC_MAX_ROWS
 
 
@@ -74,6 +74,8 @@ def _load():
     lib.losa_free.restype = None
     lib.losa_check_status.argtypes = [vp]
     lib.losa_check_status.restype = i32
+    lib.losa_exp2_eval.argtypes = [vp, vp, i64, vp]
+    lib.losa_exp2_eval.restype = i32
     lib.losa_strerror.argtypes = [i32]
     lib.losa_strerror.restype = ctypes.c_char_p
     lib.losa_version.argtypes = []
@@ -225,6 +227,16 @@ def sparse_attn(q, k, v, L, pattern: Pattern, scale=None, out_dtype=torch.float3
                                _stream(stream))
     _check("losa_sparse_attn", st)
     return o, lse
+
+
+def exp2_eval(x, stream=None):
+    """2^x with the kernels' FMA-pipe exponential (diagnostic)."""
+    if not (x.is_cuda and x.is_contiguous() and x.dtype == torch.float32):
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check("losa_exp2_eval", _lib.losa_exp2_eval(x.data_ptr(), y.data_ptr(), x.numel(),
+                                                 _stream(stream)))
+    return y
 
 
 def check_status(stream=None):

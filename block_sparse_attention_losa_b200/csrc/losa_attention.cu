@@ -74,7 +74,25 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
   }
 }
 
+__global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                 int64_t n) {
+  for (int64_t i = 2 * (blockIdx.x * int64_t(blockDim.x) + threadIdx.x); i < n;
+       i += 2 * int64_t(gridDim.x) * blockDim.x) {
+    float y0, y1;
+    exp2_fma2(x[i], i + 1 < n ? x[i + 1] : 0.f, y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_eval(const float* x, float* y, int64_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int grid = int(std::min<int64_t>((n / 2 + 255) / 256 + 1, 148 * 8));
+  exp2_eval_kernel<<<grid, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {
   // n is a multiple of 64 (d in {64, 128}); 16-byte aligned pointers.

@@ -81,6 +81,12 @@ struct AttnLayout {
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
 };
 
+// Of every 16 column pairs, how many take exp2 on the FMA pipe (the rest
+// use MUFU ex2): a small share where the softmax is also issue-bound (flash
+// pass, sparse step), a large one in the mass pass, which is MUFU-bound.
+constexpr int kPolyPairsFlash = 0;
+constexpr int kPolyPairsMass = 7;
+
 constexpr int kAttnThreads = 384;
 constexpr int kAttnLaunchRegs = 168;   // checked against ptxas at build time
 constexpr int kSoftmaxRegs = 216;
@@ -420,15 +426,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int sc = 0;              // S_t completions seen
     bool ok = true;
 
+    // List entries run one iteration ahead: those of iteration j + 1 are
+    // fetched at the top of iteration j, so their global-load latency hides
+    // behind a whole iteration. Past the end of the list: 0 (all rows off).
+    int ent_next[EPI];
+    if constexpr (!kDense) {
+#pragma unroll
+      for (int e = 0; e < EPI; ++e)
+        ent_next[e] = (e < n) ? __ldg(p.tile_entry + e_begin[t] + e) : 0;
+    }
     for (int j = 0; j < n_iter; ++j) {
-      // The list entries of this iteration: fetched before waiting for S so
-      // the global-load latency hides behind the wait. Past the end: off.
       int ent[EPI];
       if constexpr (!kDense) {
 #pragma unroll
         for (int e = 0; e < EPI; ++e) {
-          const int idx = j * EPI + e;
-          ent[e] = (idx < n) ? __ldg(p.tile_entry + e_begin[t] + idx) : 0;
+          ent[e] = ent_next[e];
+          const int idx = (j + 1) * EPI + e;
+          ent_next[e] = (idx < n) ? __ldg(p.tile_entry + e_begin[t] + idx) : 0;
         }
       }
       if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
@@ -527,9 +541,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int col = c * 32 + g * 8 + 2 * i;
-            float a0, a1;
+            float a0, a1, e0, e1;
             f2_split(f2_fma(f2_make(s[col], s[col + 1]), sl2x2, ns2), a0, a1);
-            const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+            if (((col >> 1) & 15) < kPolyPairsFlash) {
+              exp2_fma2(a0, a1, e0, e1);
+            } else {
+              e0 = ex2_approx(a0);
+              e1 = ex2_approx(a1);
+            }
             ts2[i & 1] = f2_add(ts2[i & 1], f2_make(e0, e1));
             pk[g * 4 + i] = pack_bf16x2(e0, e1);
             lbs[i] = add_bf16x2_to(lbs[i], pk[g * 4 + i]);
@@ -633,9 +652,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             f32x2 acc[2] = {0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-              float a0, a1;
+              float a0, a1, e0, e1;
               f2_split(f2_fma(f2_make(s[g * 32 + c], s[g * 32 + c + 1]), sl2x2, nl2), a0, a1);
-              acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_make(ex2_approx(a0), ex2_approx(a1)));
+              if ((c >> 1) < kPolyPairsMass) {
+                exp2_fma2(a0, a1, e0, e1);
+              } else {
+                e0 = ex2_approx(a0);
+                e1 = ex2_approx(a1);
+              }
+              acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_make(e0, e1));
             }
             part[g] = f2_sum(acc[0]) + f2_sum(acc[1]);
           }

@@ -298,6 +298,41 @@ __device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t w) {
   return acc;
 }
 
+// ---- exp2 on the FMA pipe, for two values at once (relieves MUFU).
+// Cody-Waite range reduction: x = n + f, n = round(x), f in [-1/2, 1/2];
+// 2^x = 2^n * P(f) with P the degree-5 minimax polynomial for 2^f fitted by
+// fit_exp2_poly.py (relative error 3.1e-7 in fp32 Horner form). 2^n is added
+// straight into P's exponent bits. x is clamped at -125 so 2^n stays a
+// normal number: arguments below give ~2e-38 instead of 0, far below any
+// sum this library forms.
+constexpr float kExp2C0 = 1.0000001192092896f;
+constexpr float kExp2C1 = 0.6931476593017578f;
+constexpr float kExp2C2 = 0.2402215152978897f;
+constexpr float kExp2C3 = 0.05549462139606476f;
+constexpr float kExp2C4 = 0.009673796594142914f;
+constexpr float kExp2C5 = 0.001370798796415329f;
+constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23: x + magic rounds x to an integer
+
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& y1) {
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const f32x2 x = f2_make(x0, x1);
+  const f32x2 t = f2_add(x, f2_make(kRoundMagic, kRoundMagic));   // n in the low mantissa bits
+  const f32x2 n = f2_add(t, f2_make(-kRoundMagic, -kRoundMagic));
+  const f32x2 f = f2_fma(n, f2_make(-1.f, -1.f), x);              // x - n
+  f32x2 q = f2_fma(f2_make(kExp2C5, kExp2C5), f, f2_make(kExp2C4, kExp2C4));
+  q = f2_fma(q, f, f2_make(kExp2C3, kExp2C3));
+  q = f2_fma(q, f, f2_make(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_make(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_make(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_split(q, q0, q1);
+  f2_split(t, t0, t1);
+  // t's bits are 0x4B400000 + n; shifted left by 23 only n << 23 survives.
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 // Sum of the two bf16 values packed in a 32-bit word, in fp32 (exact
 // widening of each half).
 __device__ __forceinline__ float bf16x2_sum(uint32_t w) {

@@ -226,6 +226,16 @@ void losa_free(losa_pattern* p);
  */
 int losa_check_status(void* stream);
 
+/*
+ * losa_exp2_eval - diagnostic: y[i] = 2^x[i] computed with the FMA-pipe
+ * exponential the attention kernels use for part of their softmax
+ * exponentials (Cody-Waite range reduction and a degree-5 minimax
+ * polynomial; relative error below 4e-7 for x in [-125, 127]; x below -125
+ * gives a value under 3e-38). x, y: n fp32 device values. Stream-ordered.
+ * Returns LOSA_ERR_ARG for null pointers or n < 0.
+ */
+int losa_exp2_eval(const float* x, float* y, int64_t n, void* stream);
+
 /* Short English text for a status code. Never NULL. */
 const char* losa_strerror(int status);
 
