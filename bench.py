@@ -61,6 +61,10 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ncu-case", action="store_true",
                     help="only run dense_mass x2, select, sparse_attn x2 (profiling)")
+    ap.add_argument("--tau-sweep", action="store_true",
+                    help="per tau: kept fraction, sparse vs dense time, output error vs dense")
+    ap.add_argument("--stability", action="store_true",
+                    help="frozen pattern vs fresh selections over the drifted steps")
     return ap.parse_args()
 
 
@@ -270,6 +274,120 @@ def reference_arm(args, world, rank):
     return 0
 
 
+# ------------------------------------------------------------------ analyses
+
+def _event_ms(fn, n=5, warm=2):
+    for _ in range(warm):
+        fn()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        fn()
+    z.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(z) / n
+
+
+def _full_pattern(losa, B, H, n, b, device):
+    """A pattern that keeps every block (uniform masses, tau = 1): the
+    sparse kernel then computes dense attention, the reference point for
+    sparse-vs-dense time and error."""
+    mass = torch.full((B, H, n, n), 1.0 / n, device=device, dtype=torch.float32)
+    pat = losa.select(mass, b, 1.0)
+    assert pat.nnz == B * H * n * n
+    return pat
+
+
+def tau_sweep(losa, wl, args, dev):
+    """Threshold sweep (the Wan2.1-14B-shaped workload's description): for
+    each tau, the kept-block fraction, the sparse step's time against dense
+    attention of the same kernel, and the sparse output's error against the
+    dense output on the same (drifted) inputs. One JSON line per tau."""
+    L, Lp, b, d = wl.seq_len, wl.seq_pad, wl.block, wl.head_dim
+    B, H, n = wl.batch, wl.heads, wl.n_blocks
+    qkv0 = W.generate(wl, device=dev)
+    t_con = _event_ms(lambda: losa.dense_mass(*qkv0, L, b, out_dtype=torch.bfloat16), n=3, warm=1)
+    _, _, mass = losa.dense_mass(*qkv0, L, b, out_dtype=torch.bfloat16)
+    qkv1 = W.drift(wl, qkv0, step=1, device=dev)
+    del qkv0
+    full = _full_pattern(losa, B, H, n, b, dev)
+    o_bf = torch.empty(B, H, Lp, d, device=dev, dtype=torch.bfloat16)
+    t_dense = _event_ms(lambda: losa.sparse_attn(*qkv1, L, full, out_dtype=torch.bfloat16,
+                                                 o=o_bf, want_lse=False))
+    o_dense, _ = losa.sparse_attn(*qkv1, L, full, out_dtype=torch.float32, want_lse=False)
+    f_dense = 4.0 * b * b * d * full.nnz
+    full.close()
+    peaks, _ = load_peaks()
+    out = []
+    for tau in wl.taus:
+        pat = losa.select(mass, b, tau)
+        t_sp = _event_ms(lambda: losa.sparse_attn(*qkv1, L, pat, out_dtype=torch.bfloat16,
+                                                  o=o_bf, want_lse=False))
+        o_sp, _ = losa.sparse_attn(*qkv1, L, pat, out_dtype=torch.float32, want_lse=False)
+        diff = (o_sp[:, :, :L] - o_dense[:, :, :L]).abs()
+        f_sp = 4.0 * b * b * d * pat.nnz
+        rec = {"analysis": "tau_sweep", "workload": wl.name, "tau": tau,
+               "kept_fraction": pat.density(), "retained_blocks": pat.nnz,
+               "tile_overhead": pat.tile_entries * (128 // b) / pat.nnz,
+               "sparse_ms": t_sp, "dense_ms": t_dense, "speedup_vs_dense": t_dense / t_sp,
+               "sparse_tflops_retained": f_sp / (t_sp * 1e-3) / 1e12,
+               "dense_tflops": f_dense / (t_dense * 1e-3) / 1e12,
+               "frac_of_peak": f_sp / (t_sp * 1e-3) / 1e12 / peaks["bf16_tflops"],
+               "err_max_vs_dense": diff.max().item(), "err_mean_vs_dense": diff.mean().item(),
+               "err_rel_fro_vs_dense": (torch.linalg.vector_norm(o_sp[:, :, :L] - o_dense[:, :, :L])
+                                        / torch.linalg.vector_norm(o_dense[:, :, :L])).item(),
+               "construction_ms": t_con}
+        pat.close()
+        print(json.dumps(rec), flush=True)
+        out.append(rec)
+    return out
+
+
+def stability(losa, wl, args, dev, tau=0.99):
+    """The pages' second observation (the high-mass support stays stable
+    across denoising steps): freeze the pattern at the construction step,
+    then at every later (drifted) step measure the mass the frozen blocks
+    still hold under that step's exact masses, and how many of a fresh
+    selection's blocks the frozen pattern covers. One JSON line per step."""
+    L, b = wl.seq_len, wl.block
+    B, H, n = wl.batch, wl.heads, wl.n_blocks
+    R = B * H * n
+    qkv = W.generate(wl, device=dev)
+    _, _, mass0 = losa.dense_mass(*qkv, L, b, out_dtype=torch.bfloat16)
+    pat0 = losa.select(mass0, b, tau)
+    ex0 = pat0.export()
+    rows0 = torch.repeat_interleave(torch.arange(R, device=dev),
+                                    (ex0["row_ptr"][1:] - ex0["row_ptr"][:-1]).long())
+    keep0 = torch.zeros(R, n, dtype=torch.bool, device=dev)
+    keep0[rows0, ex0["col_idx"].long()] = True
+    steps = max(1, wl.sparse_steps or 10)
+    out = []
+    for s in range(1, steps + 1):
+        qkv = W.drift(wl, qkv, step=s, device=dev)
+        _, _, mass_s = losa.dense_mass(*qkv, L, b, out_dtype=torch.bfloat16)
+        m = mass_s.view(R, n).double()
+        held = (m * keep0).sum(dim=1)
+        pat_s = losa.select(mass_s, b, tau)
+        ex_s = pat_s.export()
+        rows_s = torch.repeat_interleave(torch.arange(R, device=dev),
+                                         (ex_s["row_ptr"][1:] - ex_s["row_ptr"][:-1]).long())
+        keep_s = torch.zeros(R, n, dtype=torch.bool, device=dev)
+        keep_s[rows_s, ex_s["col_idx"].long()] = True
+        inter = (keep0 & keep_s).sum().item()
+        rec = {"analysis": "stability", "workload": wl.name, "step": s, "tau": tau,
+               "frozen_mass_min": held.min().item(), "frozen_mass_mean": held.mean().item(),
+               "rows_reaching_tau": (held >= tau).double().mean().item(),
+               "recall_of_fresh": inter / max(1, keep_s.sum().item()),
+               "jaccard": inter / max(1, (keep0 | keep_s).sum().item()),
+               "kept_frozen": pat0.density(), "kept_fresh": pat_s.density()}
+        pat_s.close()
+        print(json.dumps(rec), flush=True)
+        out.append(rec)
+    pat0.close()
+    return out
+
+
 # ------------------------------------------------------------------ LoSA arm
 
 def main():
@@ -284,6 +402,13 @@ def main():
     import block_sparse_attention_losa_b200 as losa
 
     wl = W.WORKLOADS[args.workload]
+    if args.tau_sweep or args.stability:
+        dev = torch.device("cuda", local)
+        if args.tau_sweep:
+            tau_sweep(losa, wl, args, dev)
+        if args.stability:
+            stability(losa, wl, args, dev)
+        return 0
     n_sparse = args.sparse_steps if args.sparse_steps is not None else max(1, wl.sparse_steps)
     if args.ncu_case:
         n_sparse = 1  # keeps the device footprint of a profiled run small
@@ -291,12 +416,17 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
 
-    # Inputs: construction Q/K/V plus n_sparse drifted sets, all resident.
+    # Inputs: construction Q/K/V plus the drifted sets of the sparse steps,
+    # all resident. At most ~16 GB of distinct drifted sets are kept; longer
+    # runs (HunyuanVideo-shaped: 40 steps) cycle through them.
     qkv0 = W.generate(wl, device=dev)
-    sets, prev = [], qkv0
-    for s in range(n_sparse):
+    set_bytes = 3 * wl.batch * wl.heads * Lp * d * 2
+    n_sets = max(1, min(n_sparse, int(16e9 // set_bytes)))
+    distinct, prev = [], qkv0
+    for s in range(n_sets):
         prev = W.drift(wl, prev, step=s + 1, device=dev)
-        sets.append(prev)
+        distinct.append(prev)
+    sets = [distinct[s % n_sets] for s in range(n_sparse)]
     B, H = wl.batch, wl.heads
     o_dense = torch.empty(B, H, Lp, d, device=dev, dtype=torch.bfloat16)
     lse = torch.empty(B, H, Lp, device=dev, dtype=torch.float32)
@@ -382,7 +512,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": wl.name, "batch": B, "heads": H, "head_dim": d,
                    "seq_len": L, "seq_pad": Lp, "block": b, "tau": tau,
-                   "sparse_steps": n_sparse, "l2": "inputs larger than L2 (3 x "
+                   "sparse_steps": n_sparse, "distinct_step_inputs": n_sets,
+                   "l2": "inputs larger than L2 (3 x "
                    f"{B * H * Lp * d * 2 / 1e6:.0f} MB per call)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "sparse_attn": {"ms": sparse_ms, "tflops": sparse_tf, "frac_of_peak": sparse_tf / peak,

@@ -44,11 +44,11 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int L_pad, int d, int 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, int NS, bool kDense, bool kOutBf16, int BLK>
+template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK>
 cudaError_t run(const void* q, const void* k, const void* v, int BH, const AttnParams& p,
                 dim3 grid, cudaStream_t stream) {
-  using Lay = AttnLayout<D, BN, NS>;
-  auto kern = attn_kernel<D, BN, NS, kDense, kOutBf16, BLK>;
+  using Lay = AttnLayout<D, BN, NSK, NSV>;
+  auto kern = attn_kernel<D, BN, NSK, NSV, kDense, kOutBf16, BLK>;
   // Cheap, and per device: set on every launch.
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM_ALLOC);
@@ -120,16 +120,16 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, in
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
   const dim3 grid((p.n_qt + 1) / 2, BH);  // two query tiles per CTA
-#define LOSA_DENSE_CASE(D_, NS_, BLK_)                                                     \
-  if (d == D_ && block == BLK_)                                                           \
-    return out_bf16 ? run<D_, 128, NS_, true, true, BLK_>(q, k, v, BH, p, grid, stream)  \
-                    : run<D_, 128, NS_, true, false, BLK_>(q, k, v, BH, p, grid, stream);
-  LOSA_DENSE_CASE(128, 2, 128)
-  LOSA_DENSE_CASE(128, 2, 64)
-  LOSA_DENSE_CASE(128, 2, 32)
-  LOSA_DENSE_CASE(64, 4, 128)
-  LOSA_DENSE_CASE(64, 4, 64)
-  LOSA_DENSE_CASE(64, 4, 32)
+#define LOSA_DENSE_CASE(D_, NSK_, NSV_, BLK_)                                                   \
+  if (d == D_ && block == BLK_)                                                                \
+    return out_bf16 ? run<D_, 128, NSK_, NSV_, true, true, BLK_>(q, k, v, BH, p, grid, stream) \
+                    : run<D_, 128, NSK_, NSV_, true, false, BLK_>(q, k, v, BH, p, grid, stream);
+  LOSA_DENSE_CASE(128, 3, 2, 128)
+  LOSA_DENSE_CASE(128, 3, 2, 64)
+  LOSA_DENSE_CASE(128, 3, 2, 32)
+  LOSA_DENSE_CASE(64, 4, 4, 128)
+  LOSA_DENSE_CASE(64, 4, 4, 64)
+  LOSA_DENSE_CASE(64, 4, 4, 32)
 #undef LOSA_DENSE_CASE
   return cudaErrorInvalidValue;
 }
@@ -157,16 +157,16 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, in
   p.n_tiles = int(pat->n_tiles);
   const dim3 grid(unsigned((pat->n_tiles + 1) / 2));  // two tiles per CTA
   if (pat->n_tiles == 0) return cudaSuccess;
-#define LOSA_SPARSE_CASE(D_, NS_, BLK_)                                                     \
-  if (d == D_ && pat->block == BLK_)                                                       \
-    return out_bf16 ? run<D_, 128, NS_, false, true, BLK_>(q, k, v, BH, p, grid, stream)  \
-                    : run<D_, 128, NS_, false, false, BLK_>(q, k, v, BH, p, grid, stream);
-  LOSA_SPARSE_CASE(128, 2, 128)
-  LOSA_SPARSE_CASE(128, 2, 64)
-  LOSA_SPARSE_CASE(128, 2, 32)
-  LOSA_SPARSE_CASE(64, 4, 128)
-  LOSA_SPARSE_CASE(64, 4, 64)
-  LOSA_SPARSE_CASE(64, 4, 32)
+#define LOSA_SPARSE_CASE(D_, NSK_, NSV_, BLK_)                                                   \
+  if (d == D_ && pat->block == BLK_)                                                            \
+    return out_bf16 ? run<D_, 128, NSK_, NSV_, false, true, BLK_>(q, k, v, BH, p, grid, stream) \
+                    : run<D_, 128, NSK_, NSV_, false, false, BLK_>(q, k, v, BH, p, grid, stream);
+  LOSA_SPARSE_CASE(128, 3, 2, 128)
+  LOSA_SPARSE_CASE(128, 3, 2, 64)
+  LOSA_SPARSE_CASE(128, 3, 2, 32)
+  LOSA_SPARSE_CASE(64, 4, 4, 128)
+  LOSA_SPARSE_CASE(64, 4, 4, 64)
+  LOSA_SPARSE_CASE(64, 4, 4, 32)
 #undef LOSA_SPARSE_CASE
   return cudaErrorInvalidValue;
 }

@@ -52,7 +52,7 @@ struct AttnParams {
   int* status;
 };
 
-template <int D, int BN, int NS>
+template <int D, int BN, int NSK, int NSV>
 struct AttnLayout {
   static constexpr int BM = 128;
   static constexpr int NT = 2;                           // query tiles per CTA
@@ -60,11 +60,11 @@ struct AttnLayout {
   static constexpr int KV_BYTES = BN * D * 2;            // D/64 slabs of BN*128 B
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-  // q_full[2], k_full/k_empty/v_full/v_empty[NS], s_full[2], s_free[2],
+  static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
+  // q_full[2], k_full/k_empty[NSK], v_full/v_empty[NSV], s_full[2], s_free[2],
   // p_full[2], o_full[2], red_bar[2][2], drain
-  static constexpr int N_BARS = 2 + 4 * NS + 8 + 4 + 1;
+  static constexpr int N_BARS = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem addr, abort flag
   static constexpr int OFF_RED = OFF_MISC + 16;          // float red[2 tiles][2][4 warps][4]
   static constexpr int BYTES = OFF_RED + 2 * 2 * 4 * 4 * 4;
@@ -82,10 +82,11 @@ struct AttnLayout {
 };
 
 // Of every 16 column pairs, how many take exp2 on the FMA pipe (the rest
-// use MUFU ex2): a small share where the softmax is also issue-bound (flash
-// pass, sparse step), a large one in the mass pass, which is MUFU-bound.
-constexpr int kPolyPairsFlash = 0;
-constexpr int kPolyPairsMass = 7;
+// use MUFU ex2). Measured on B200: the flash softmax (both head dims) is
+// not limited by MUFU throughput, so moving work to the FMA pipe only adds
+// instructions there; the mass pass is, and gains from moving 7 of 16.
+template <int D> constexpr int poly_pairs_flash() { return 0; }
+template <int D> constexpr int poly_pairs_mass() { return 7; }
 
 constexpr int kAttnThreads = 384;
 constexpr int kAttnLaunchRegs = 168;   // checked against ptxas at build time
@@ -99,11 +100,11 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kAttnThreads * kAtt
 // the mass pass sums over b x b blocks. Sparse: each 128-key iteration packs
 // EPI = BN / b consecutive entries of the tile's list into one K/V stage
 // (one b-row box each, stacked), so the tensor core always runs N = 128.
-template <int D, int BN, int NS, bool kDense, bool kOutBf16, int BLK>
+template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using Lay = AttnLayout<D, BN, NS>;
+  using Lay = AttnLayout<D, BN, NSK, NSV>;
   constexpr int BM = Lay::BM;
   constexpr int N_SLABS = D / 64;
   constexpr int BOX = kDense ? BN : BLK;  // key rows per TMA box
@@ -120,11 +121,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sV = smem + Lay::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* q_full = bars;             // [2]
-  uint64_t* k_full = q_full + 2;       // [NS]
-  uint64_t* k_empty = k_full + NS;     // [NS]
-  uint64_t* v_full = k_empty + NS;     // [NS]
-  uint64_t* v_empty = v_full + NS;     // [NS]
-  uint64_t* s_full = v_empty + NS;     // [2] MMA -> softmax t: S_t ready
+  uint64_t* k_full = q_full + 2;       // [NSK]
+  uint64_t* k_empty = k_full + NSK;    // [NSK]
+  uint64_t* v_full = k_empty + NSK;    // [NSV]
+  uint64_t* v_empty = v_full + NSV;    // [NSV]
+  uint64_t* s_full = v_empty + NSV;    // [2] MMA -> softmax t: S_t ready
   uint64_t* s_free = s_full + 2;       // [2] softmax t -> MMA: S_t read (pass 2)
   uint64_t* p_full = s_free + 2;       // [2] softmax t -> MMA: P_t in TMEM
   uint64_t* o_full = p_full + 2;       // [2] MMA -> softmax t: last PV_t done
@@ -173,9 +174,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&red_bar[2 * t], 128);
       mbar_init(&red_bar[2 * t + 1], 128);
     }
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
@@ -210,8 +213,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = true;
       // One stage = BN keys = EPI boxes of BLK rows, stacked in each slab.
       auto load_k = [&](const int (&key_row)[EPI], int head) -> bool {
-        const int ks = kc % NS;
-        if (!mbar_wait(&k_empty[ks], ((kc / NS) & 1) ^ 1, wc)) return false;
+        const int ks = kc % NSK;
+        if (!mbar_wait(&k_empty[ks], ((kc / NSK) & 1) ^ 1, wc)) return false;
         mbar_arrive_expect_tx(&k_full[ks], Lay::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < N_SLABS; ++s)
@@ -223,8 +226,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return true;
       };
       auto load_v = [&](const int (&key_row)[EPI], int head) -> bool {
-        const int vs = vc % NS;
-        if (!mbar_wait(&v_empty[vs], ((vc / NS) & 1) ^ 1, wc)) return false;
+        const int vs = vc % NSV;
+        if (!mbar_wait(&v_empty[vs], ((vc / NSV) & 1) ^ 1, wc)) return false;
         mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < N_SLABS; ++s)
@@ -266,8 +269,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // CTA releases its shared memory.
         mbar_wait_drain(&q_full[0], 0);
         mbar_wait_drain(&q_full[1], 0);
-        for (int i = (kc > NS ? kc - NS : 0); i < kc; ++i) mbar_wait_drain(&k_full[i % NS], (i / NS) & 1);
-        for (int i = (vc > NS ? vc - NS : 0); i < vc; ++i) mbar_wait_drain(&v_full[i % NS], (i / NS) & 1);
+        for (int i = (kc > NSK ? kc - NSK : 0); i < kc; ++i) mbar_wait_drain(&k_full[i % NSK], (i / NSK) & 1);
+        for (int i = (vc > NSV ? vc - NSV : 0); i < vc; ++i) mbar_wait_drain(&v_full[i % NSV], (i / NSV) & 1);
       }
     }
   } else if (warp == 9) {
@@ -301,8 +304,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return true;
       };
       auto wait_k = [&](int& ks) -> bool {
-        ks = kc % NS;
-        return mbar_wait(&k_full[ks], (kc / NS) & 1, wc);
+        ks = kc % NSK;
+        return mbar_wait(&k_full[ks], (kc / NSK) & 1, wc);
       };
       auto release_k = [&](int ks) {
         umma_commit(&k_empty[ks]);
@@ -323,8 +326,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return true;
       };
       auto wait_v = [&](int& vs) -> bool {
-        vs = vc % NS;
-        return mbar_wait(&v_full[vs], (vc / NS) & 1, wc);
+        vs = vc % NSV;
+        return mbar_wait(&v_full[vs], (vc / NSV) & 1, wc);
       };
       auto release_v = [&](int vs) {
         umma_commit(&v_empty[vs]);
@@ -543,7 +546,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int col = c * 32 + g * 8 + 2 * i;
             float a0, a1, e0, e1;
             f2_split(f2_fma(f2_make(s[col], s[col + 1]), sl2x2, ns2), a0, a1);
-            if (((col >> 1) & 15) < kPolyPairsFlash) {
+            if (((col >> 1) & 15) < poly_pairs_flash<D>()) {
               exp2_fma2(a0, a1, e0, e1);
             } else {
               e0 = ex2_approx(a0);
@@ -654,7 +657,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int c = 0; c < 32; c += 2) {
               float a0, a1, e0, e1;
               f2_split(f2_fma(f2_make(s[g * 32 + c], s[g * 32 + c + 1]), sl2x2, nl2), a0, a1);
-              if ((c >> 1) < kPolyPairsMass) {
+              if ((c >> 1) < poly_pairs_mass<D>()) {
                 exp2_fma2(a0, a1, e0, e1);
               } else {
                 e0 = ex2_approx(a0);
