@@ -232,7 +232,8 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -245,7 +246,7 @@ def reference_arm(args, world, rank):
         return 0
     wl = W.WORKLOADS[args.workload]
     n_sparse = args.sparse_steps if args.sparse_steps is not None else max(1, wl.sparse_steps)
-    per_step = max(1.0, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
+    per_step = min(args.cpu_seconds, max(1.0, min(8.0, 120.0 / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
         oracle_sample(wl, args.tau, n_sparse, per_step / 4)
     tot_f, tot_s, tot_b, threads = 0.0, 0.0, 0, os.cpu_count()

@@ -29,7 +29,7 @@ STATUS = {0: "LOSA_OK", -1: "LOSA_ERR_ARG", -2: "LOSA_ERR_CUDA", -3: "LOSA_ERR_N
 # Every symbol include/losa.h declares.
 EXPORTS = ("losa_dense_mass", "losa_select", "losa_pattern_info", "losa_pattern_export",
            "losa_select_noalloc", "losa_sparse_attn", "losa_free", "losa_check_status",
-           "losa_exp2_eval", "losa_strerror", "losa_version")
+           "losa_selftest_wait", "losa_exp2_eval", "losa_strerror", "losa_version")
 NOALLOC_MAX_ROWS = 65536  # LOSA_NOALLOC_MAX_ROWS
 
 
@@ -74,6 +74,8 @@ def _load():
     lib.losa_free.restype = None
     lib.losa_check_status.argtypes = [vp]
     lib.losa_check_status.restype = i32
+    lib.losa_selftest_wait.argtypes = [i64, vp]
+    lib.losa_selftest_wait.restype = i32
     lib.losa_exp2_eval.argtypes = [vp, vp, i64, vp]
     lib.losa_exp2_eval.restype = i32
     lib.losa_strerror.argtypes = [i32]

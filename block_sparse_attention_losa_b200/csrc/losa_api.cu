@@ -250,6 +250,13 @@ int losa_check_status(void* stream) {
   return LOSA_OK;
 }
 
+int losa_selftest_wait(int64_t limit_cycles, void* stream) {
+  if (limit_cycles <= 0 || limit_cycles > (int64_t(1) << 33)) return LOSA_ERR_ARG;
+  return launch_wait_selftest(limit_cycles, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LOSA_OK
+             : LOSA_ERR_CUDA;
+}
+
 int losa_exp2_eval(const float* x, float* y, int64_t n, void* stream) {
   if (!x || !y || n < 0) return LOSA_ERR_ARG;
   return launch_exp2_eval(x, y, n, static_cast<cudaStream_t>(stream)) == cudaSuccess

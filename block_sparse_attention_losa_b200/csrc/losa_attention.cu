@@ -85,7 +85,32 @@ __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict_
   }
 }
 
+// One bounded wait on an mbarrier nothing ever completes: it runs out after
+// `limit` SM cycles, raises the status word and returns (diagnostic of the
+// wait machinery every attention kernel uses).
+__global__ void wait_selftest_kernel(int* status, long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx wc{&abort_flag, status, limit};
+    mbar_wait(&bar, 0, wc);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(long long limit_cycles, cudaStream_t stream) {
+  int* status = device_status_word();
+  if (!status) return cudaErrorInvalidDevice;
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_cycles);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_exp2_eval(const float* x, float* y, int64_t n, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;

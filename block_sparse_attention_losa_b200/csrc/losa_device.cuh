@@ -59,6 +59,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 struct WaitCtx {
   volatile int* abort_flag;  // shared memory
   int* status;               // global device status word
+  long long limit = kWaitLimitCycles;  // SM cycles before a wait gives up
 };
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
@@ -68,7 +69,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*w.abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > w.limit) {
         *w.abort_flag = 1;
         atomicCAS(w.status, kStatusOk, kStatusTimeout);
         return false;

@@ -50,6 +50,9 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, in
                           float scale, const losa_pattern* p, void* o, bool out_bf16,
                           float* lse, cudaStream_t stream);
 
+// One bounded mbarrier wait that must run out (diagnostic).
+cudaError_t launch_wait_selftest(long long limit_cycles, cudaStream_t stream);
+
 // y = 2^x with the FMA-pipe exp2 of the attention kernels (diagnostic).
 cudaError_t launch_exp2_eval(const float* x, float* y, int64_t n, cudaStream_t stream);
 

@@ -227,6 +227,17 @@ void losa_free(losa_pattern* p);
 int losa_check_status(void* stream);
 
 /*
+ * losa_selftest_wait - diagnostic of the failure path every kernel uses:
+ * launches one wait on a barrier that nothing completes. The wait gives up
+ * after limit_cycles SM cycles (0 < limit_cycles <= 2^33), records a
+ * timeout in the device status word and the kernel returns normally, so the
+ * CUDA context stays usable; the next losa_check_status on that stream
+ * returns LOSA_ERR_TIMEOUT and clears the word. Returns LOSA_ERR_ARG for a
+ * limit out of range.
+ */
+int losa_selftest_wait(int64_t limit_cycles, void* stream);
+
+/*
  * losa_exp2_eval - diagnostic: y[i] = 2^x[i] computed with the FMA-pipe
  * exponential the attention kernels use for part of their softmax
  * exponentials (Cody-Waite range reduction and a degree-5 minimax

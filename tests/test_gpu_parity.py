@@ -287,3 +287,23 @@ def test_fma_pipe_exp2_error_bound(losa):
     assert rel.max().item() < 4e-7, rel.max().item()
     low = losa.exp2_eval(torch.tensor([-126.0, -300.0, float("-inf")]).cuda()).cpu()
     assert torch.all(low >= 0).item() and torch.all(low < 3e-38).item()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(losa):
+    """A wait nothing completes gives up after its limit (here ~1 ms of SM
+    cycles), the status word reports it once, and the device keeps working."""
+    lib = losa.lib()
+    losa.check_status()                      # start clean
+    assert lib.losa_selftest_wait(2_000_000, None) == 0
+    with pytest.raises(losa.LosaError) as e:
+        losa.check_status(torch.cuda.default_stream())
+    assert e.value.status == -4              # LOSA_ERR_TIMEOUT
+    losa.check_status()                      # cleared
+    assert lib.losa_selftest_wait(0, None) == -1
+    # the context is still usable: a normal call after the timeout
+    wl = W.custom("after_timeout", 1, 64, (2, 8, 8), 32, amplitude=1.0, seed=2)
+    q, k, v = (t.cuda() for t in W.generate(wl, dtype=torch.bfloat16))
+    o, lse, mass = losa.dense_mass(q, k, v, wl.seq_len, wl.block)
+    torch.cuda.synchronize()
+    losa.check_status()
+    assert torch.allclose(mass.sum(-1), torch.ones_like(mass.sum(-1)), atol=1e-4)
