@@ -288,17 +288,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// acc + (both bf16 halves of w), each widened exactly to fp32.
-__device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t w) {
-  asm("{\n\t.reg .b16 lo, hi;\n\t"
-      "mov.b32 {lo, hi}, %1;\n\t"
-      "add.f32.bf16 %0, lo, %0;\n\t"
-      "add.f32.bf16 %0, hi, %0;\n\t}"
-      : "+f"(acc)
-      : "r"(w));
-  return acc;
-}
-
 // ---- exp2 on the FMA pipe, for two values at once (relieves MUFU).
 // Cody-Waite range reduction: x = n + f, n = round(x), f in [-1/2, 1/2];
 // 2^x = 2^n * P(f) with P the degree-5 minimax polynomial for 2^f fitted by
@@ -332,12 +321,6 @@ __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& 
   // t's bits are 0x4B400000 + n; shifted left by 23 only n << 23 survives.
   y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
-// Sum of the two bf16 values packed in a 32-bit word, in fp32 (exact
-// widening of each half).
-__device__ __forceinline__ float bf16x2_sum(uint32_t w) {
-  return __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
