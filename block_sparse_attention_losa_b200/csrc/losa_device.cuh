@@ -323,8 +323,5 @@ __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& 
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 }  // namespace losa
