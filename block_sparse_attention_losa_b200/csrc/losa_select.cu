@@ -6,12 +6,11 @@
 // and query block, the smallest key/value block set meeting the threshold").
 //
 // All of it is integer work on 64-bit fixed-point masses x = round(m * 2^48),
-// so the result is bit-exact. Instead of sorting each row, the kernel finds
-// the cut with an MSD radix select over the sort keys
+// so the result is bit-exact. Each row's sort keys
 //     key(J) = ((2^49 - 1 - x_J) << 11) | J          (< 2^60, unique per row)
-// whose ascending order is (x desc, J asc): it narrows 8 bits at a time to
-// the bucket where the running sum first reaches the threshold, keeping
-// per-bucket sums and counts in shared memory. The kept set is then
+// ascend in (x desc, J asc) order; a bitonic sort in shared memory orders
+// them, a block prefix scan accumulates the masses in that order, and the
+// cut is the first prefix that reaches the threshold. The kept set is then
 // {J : key(J) <= cut key}, written out in ascending J.
 #include <cub/block/block_reduce.cuh>
 #include <cub/block/block_scan.cuh>
@@ -27,9 +26,7 @@ namespace losa {
 namespace {
 
 constexpr int kSelThreads = 256;
-constexpr int kMaxBlocks = 2047;                               // n <= 2047: J fits 11 bits
-constexpr int kKeysPerThread = (kMaxBlocks + kSelThreads) / kSelThreads;  // 8
-constexpr unsigned long long kXMax = (1ull << 49) - 1;          // masses in [0, 2)
+constexpr unsigned long long kXMax = (1ull << 49) - 1;          // masses in [0, 2); J < 2048
 constexpr unsigned long long kNoKey = ~0ull;
 
 // x = round(m * 2^48) (ties to even; exact, as m * 2^48 only shifts the
@@ -54,132 +51,109 @@ __device__ __forceinline__ bool reaches(unsigned long long C, unsigned long long
 }
 
 // One CTA per row: the cut key, kept count, kept and total fixed-point mass.
+// The row's sort keys are sorted ascending in shared memory with a bitonic
+// network (NP = n rounded up to a power of two, padded with keys that sort
+// last), the fixed-point masses are prefix-summed in that order, and the cut
+// is the first position k where 2^48 * C_k >= tau_fx * S (exact, 128-bit).
+// No atomics, so the result does not depend on scheduling.
+template <int NP>
 __global__ void __launch_bounds__(kSelThreads)
     select_cut_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
                       unsigned long long* __restrict__ cut_key, int* __restrict__ count,
                       long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
                       int* status) {
-  using Reduce = cub::BlockReduce<unsigned long long, kSelThreads>;
+  constexpr int IPT = NP / kSelThreads > 0 ? NP / kSelThreads : 1;  // keys per thread
+  constexpr int NT = NP / IPT;                                       // threads holding keys
+  using Scan = cub::BlockScan<unsigned long long, kSelThreads>;
+  using Reduce = cub::BlockReduce<int, kSelThreads>;
+  __shared__ unsigned long long keys[NP];
+  __shared__ typename Scan::TempStorage scan_tmp;
   __shared__ typename Reduce::TempStorage red_tmp;
-  __shared__ unsigned long long bsum[256];
-  __shared__ unsigned int bcnt[256];
-  __shared__ unsigned long long sh_S, sh_acc, sh_hi, sh_cut;
-  __shared__ int sh_done, sh_bad;
+  __shared__ int sh_bad, sh_k;
 
   const int row = blockIdx.x;
   const float* mrow = mass + size_t(row) * n;
-  unsigned long long key[kKeysPerThread];
-  long long xs[kKeysPerThread];
+  if (threadIdx.x == 0) sh_bad = 0;
+  __syncthreads();
   bool bad = false;
-  unsigned long long local = 0;
-#pragma unroll
-  for (int i = 0; i < kKeysPerThread; ++i) {
-    const int J = threadIdx.x + i * kSelThreads;
-    key[i] = kNoKey;
-    xs[i] = 0;
+  for (int J = threadIdx.x; J < NP; J += kSelThreads) {
+    unsigned long long key = kNoKey;
     if (J < n) {
       long long x;
       bad |= !to_fixed(mrow[J], x);
-      xs[i] = x;
-      key[i] = sort_key(x, J);
-      local += (unsigned long long)x;
+      key = sort_key(x, J);
+    }
+    keys[J] = key;
+  }
+  if (bad) sh_bad = 1;
+  // Bitonic sort, ascending.
+  for (int size = 2; size <= NP; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int pr = threadIdx.x; pr < NP / 2; pr += kSelThreads) {
+        const int i = 2 * stride * (pr / stride) + (pr % stride);
+        const int k = i + stride;
+        const unsigned long long a = keys[i], b = keys[k];
+        const bool up = (i & size) == 0;
+        if ((a > b) == up) {
+          keys[i] = b;
+          keys[k] = a;
+        }
+      }
     }
   }
-  if (threadIdx.x == 0) sh_bad = 0;
   __syncthreads();
-  if (bad) sh_bad = 1;
-  const unsigned long long S_part = Reduce(red_tmp).Sum(local);
+  // Fixed-point masses in sorted order (thread t owns positions
+  // [t*IPT, t*IPT + IPT)); padding keys carry no mass.
+  unsigned long long xs[IPT];
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    const int pos = threadIdx.x * IPT + i;
+    const unsigned long long key = (threadIdx.x < NT) ? keys[pos] : kNoKey;
+    xs[i] = (key == kNoKey) ? 0ull : kXMax - (key >> 11);
+  }
+  unsigned long long incl[IPT], S;
+  Scan(scan_tmp).InclusiveSum(xs, incl, S);
+  // First position whose running sum reaches the threshold (k >= 1; the full
+  // row always reaches it, and an all-zero row stops at its first key).
+  int first = NP;
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    const int pos = threadIdx.x * IPT + i;
+    if (threadIdx.x < NT && pos < n && first == NP && reaches(incl[i], tau_fx, S)) first = pos;
+  }
+  const int kmin = Reduce(red_tmp).Reduce(first, cub::Min());
+  if (threadIdx.x == 0) sh_k = kmin;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    sh_S = S_part;
-    sh_acc = 0;
-    sh_hi = 0;
-    sh_done = 0;
+  const int kcut = sh_k;
+  if (threadIdx.x < NT && kcut / IPT == int(threadIdx.x)) {
+    // The thread holding the cut position writes the row's results.
+    const int i = kcut % IPT;
+    cut_key[row] = keys[kcut];
+    count[row] = kcut + 1;
+    retained_fx[row] = (long long)incl[i];
+    total_fx[row] = (long long)S;
     if (sh_bad) atomicCAS(status, kStatusOk, kStatusBadMass);
   }
-  __syncthreads();
-  const unsigned long long S = sh_S;
+}
 
-  // MSD radix select, 8 bits per pass from bit 56 down.
-  int shift = 56;
-  for (; shift >= 0; shift -= 8) {
-    bsum[threadIdx.x] = 0;
-    bcnt[threadIdx.x] = 0;
-    __syncthreads();
-    const unsigned long long hi = sh_hi;
-#pragma unroll
-    for (int i = 0; i < kKeysPerThread; ++i) {
-      if (key[i] != kNoKey && (shift == 56 || (key[i] >> (shift + 8)) == hi)) {
-        const int d = int((key[i] >> shift) & 0xFF);
-        atomicAdd(&bsum[d], (unsigned long long)xs[i]);
-        atomicAdd(&bcnt[d], 1u);
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      // Warp 0: first non-empty bucket where the running sum reaches the
-      // threshold. Lane t owns buckets [8t, 8t + 8).
-      const int t = threadIdx.x;
-      unsigned long long my = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) my += bsum[t * 8 + j];
-      unsigned long long incl = my;  // inclusive warp scan
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (t >= off) incl += v;
-      }
-      const unsigned long long acc = sh_acc;
-      unsigned long long run = acc + incl - my;  // sum of buckets before mine
-      int found = 256;
-      unsigned long long before = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int d = t * 8 + j;
-        const unsigned long long after = run + bsum[d];
-        if (found == 256 && bcnt[d] > 0 && reaches(after, tau_fx, S)) {
-          found = d;
-          before = run;
-        }
-        run = after;
-      }
-      const int first = __reduce_min_sync(0xffffffffu, unsigned(found));
-      if (found == first && found < 256) {
-        sh_acc = before;
-        sh_hi = (sh_hi << 8) | unsigned(found);
-        sh_done = (bcnt[found] == 1) ? 1 : 0;
-      }
-    }
-    __syncthreads();
-    if (sh_done) break;
+// Launches the cut kernel with the smallest power-of-two capacity >= n.
+cudaError_t launch_select_cut(const float* mass, int64_t R, int n, unsigned long long tau_fx,
+                              unsigned long long* cut, int* cnt, long long* retained,
+                              long long* total, int* status, cudaStream_t stream) {
+#define LOSA_CUT(NP_)                                                                      \
+  if (n <= NP_) {                                                                          \
+    select_cut_kernel<NP_><<<unsigned(R), kSelThreads, 0, stream>>>(mass, n, tau_fx, cut, \
+                                                                     cnt, retained, total, \
+                                                                     status);              \
+    return cudaGetLastError();                                                             \
   }
-  // The cut key: the single key left in the chosen bucket.
-  const int s_final = shift < 0 ? 0 : shift;
-  if (threadIdx.x == 0) sh_cut = kNoKey;
-  __syncthreads();
-  const unsigned long long hi = sh_hi;
-#pragma unroll
-  for (int i = 0; i < kKeysPerThread; ++i)
-    if (key[i] != kNoKey && (key[i] >> s_final) == hi) sh_cut = key[i];
-  __syncthreads();
-  const unsigned long long cut = sh_cut;
-  unsigned long long kept = 0, kept_n = 0;
-#pragma unroll
-  for (int i = 0; i < kKeysPerThread; ++i) {
-    if (key[i] <= cut) {
-      kept += (unsigned long long)xs[i];
-      kept_n += 1;
-    }
-  }
-  const unsigned long long C = Reduce(red_tmp).Sum(kept);
-  __syncthreads();
-  const unsigned long long K = Reduce(red_tmp).Sum(kept_n);
-  if (threadIdx.x == 0) {
-    cut_key[row] = cut;
-    count[row] = int(K);
-    retained_fx[row] = (long long)C;
-    total_fx[row] = (long long)S;
-  }
+  LOSA_CUT(256)
+  LOSA_CUT(512)
+  LOSA_CUT(1024)
+  LOSA_CUT(2048)
+#undef LOSA_CUT
+  return cudaErrorInvalidValue;
 }
 
 // Per 128-row tile (128/block query blocks): which key blocks each query
@@ -357,9 +331,8 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
   auto* hist = reinterpret_cast<int*>(scratch + s_hist);
   auto* cursor = reinterpret_cast<int*>(scratch + s_cur);
 
-  select_cut_kernel<<<unsigned(R), kSelThreads, 0, stream>>>(mass, n, tau_fx, cut, cnt,
-                                                              (long long*)p->retained_fx,
-                                                              (long long*)p->total_fx, status);
+  launch_select_cut(mass, R, n, tau_fx, cut, cnt, (long long*)p->retained_fx,
+                    (long long*)p->total_fx, status, stream);
   tile_count_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(mass, cut, n, qpt, n_qt, tcnt);
   scan_kernel<<<1, 1024, 0, stream>>>(cnt, int(R), p->row_ptr);
   scan_kernel<<<1, 1024, 0, stream>>>(tcnt, int(T), p->tile_ptr);
@@ -492,9 +465,8 @@ extern "C" int losa_select_noalloc(const float* mass, int B, int H, int n_blocks
   auto* cnt = reinterpret_cast<int*>(scratch + kNoallocCutBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned long long tau_fx = (unsigned long long)llrint(tau * 281474976710656.0);
-  select_cut_kernel<<<unsigned(R), kSelThreads, 0, s>>>(mass, n_blocks, tau_fx, cut, cnt,
-                                                         (long long*)retained_fx,
-                                                         (long long*)total_fx, status);
+  launch_select_cut(mass, R, n_blocks, tau_fx, cut, cnt, (long long*)retained_fx,
+                    (long long*)total_fx, status, s);
   scan_kernel<<<1, 1024, 0, s>>>(cnt, int(R), row_ptr);
   row_write_kernel<<<unsigned(R), kSelThreads, 0, s>>>(mass, n_blocks, cut, row_ptr, col_idx,
                                                        (long long)col_capacity);
