@@ -28,8 +28,9 @@ STATUS = {0: "LOSA_OK", -1: "LOSA_ERR_ARG", -2: "LOSA_ERR_CUDA", -3: "LOSA_ERR_N
 
 # Every symbol include/losa.h declares.
 EXPORTS = ("losa_dense_mass", "losa_select", "losa_pattern_info", "losa_pattern_export",
-           "losa_select_noalloc", "losa_sparse_attn", "losa_free", "losa_check_status",
-           "losa_selftest_wait", "losa_exp2_eval", "losa_strerror", "losa_version")
+           "losa_pattern_import", "losa_select_noalloc", "losa_sparse_attn", "losa_free",
+           "losa_check_status", "losa_selftest_wait", "losa_exp2_eval", "losa_strerror",
+           "losa_version")
 NOALLOC_MAX_ROWS = 65536  # LOSA_NOALLOC_MAX_ROWS
 
 
@@ -65,6 +66,9 @@ def _load():
     lib.losa_pattern_info.restype = i32
     lib.losa_pattern_export.argtypes = [vp] * 9
     lib.losa_pattern_export.restype = i32
+    lib.losa_pattern_import.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32,
+                                        ctypes.POINTER(vp), vp]
+    lib.losa_pattern_import.restype = i32
     i64 = ctypes.c_int64
     lib.losa_select_noalloc.argtypes = [vp, i32, i32, i32, f64, vp, vp, i64, vp, vp, vp]
     lib.losa_select_noalloc.restype = i32
@@ -209,6 +213,30 @@ def select(mass, block, tau=0.99, stream=None):
                           _stream(stream))
     _check("losa_select", st)
     return Pattern(h, mass.device)
+
+
+def import_pattern(row_ptr, col_idx, B, H, n_blocks, block, retained_fx=None, total_fx=None,
+                   device=None, stream=None):
+    """A Pattern from a stored host CSR (e.g. Pattern.export('cpu') of an
+    earlier selection). Arrays are converted to contiguous host int32/int64."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+        else torch.device(device)
+    host = lambda t, dt: None if t is None else \
+        torch.as_tensor(t).to("cpu", dtype=dt).contiguous()
+    rp, ci = host(row_ptr, torch.int32), host(col_idx, torch.int32)
+    rf, tf = host(retained_fx, torch.int64), host(total_fx, torch.int64)
+    R = int(B) * int(H) * int(n_blocks)
+    if rp.numel() != R + 1 or ci.numel() != int(rp[-1]) or \
+            any(t is not None and t.numel() != R for t in (rf, tf)):
+        raise ValueError("CSR array sizes do not match B * H * n_blocks")
+    ptr = lambda t: None if t is None or t.numel() == 0 else t.data_ptr()
+    h = ctypes.c_void_p()
+    with torch.cuda.device(device):
+        st = _lib.losa_pattern_import(ptr(rp), ptr(ci), ptr(rf), ptr(tf), int(B), int(H),
+                                      int(n_blocks), int(block), ctypes.byref(h),
+                                      _stream(stream))
+    _check("losa_pattern_import", st)
+    return Pattern(h, device)
 
 
 def sparse_attn(q, k, v, L, pattern: Pattern, scale=None, out_dtype=torch.float32, o=None,

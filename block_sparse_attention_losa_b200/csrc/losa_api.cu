@@ -1,8 +1,11 @@
 // losa_api.cu - the library's C ABI: argument checks, the per-device status
 // word, the fp32 entry conversion, and pattern ownership.
 #include <cmath>
+#include <algorithm>
+#include <climits>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "losa_device.cuh"
 #include "losa_internal.h"
@@ -80,6 +83,49 @@ bool valid_attn_shape(int B, int H, int L, int L_pad, int d, int block) {
   if (L_pad / block > 2047) return false;
   if (int64_t(B) * H > 65535) return false;
   return true;
+}
+
+// Checks a host CSR for losa_pattern_import: row_ptr[0] = 0, every row
+// non-empty with at most n entries, columns strictly ascending in [0, n).
+// Returns the total of the 128-row tiles' union sizes, or -1 when invalid.
+int64_t validate_csr(const int32_t* row_ptr, const int32_t* col_idx, int BH, int n,
+                     int block) {
+  const int64_t R = int64_t(BH) * n;
+  if (row_ptr[0] != 0) return -1;
+  for (int64_t r = 0; r < R; ++r) {
+    const int64_t len = int64_t(row_ptr[r + 1]) - row_ptr[r];
+    if (len < 1 || len > n) return -1;
+  }
+  const int64_t nnz = row_ptr[R];
+  if (nnz > int64_t(INT32_MAX)) return -1;
+  for (int64_t r = 0; r < R; ++r) {
+    int prev = -1;
+    for (int64_t e = row_ptr[r]; e < row_ptr[r + 1]; ++e) {
+      const int J = col_idx[e];
+      if (J <= prev || J >= n) return -1;
+      prev = J;
+    }
+  }
+  // Union sizes: a key block counts once per tile (stamped with the tile).
+  const int qpt = 128 / block;
+  const int n_qt = (n * block + 127) / 128;
+  std::vector<int64_t> stamp(size_t(n), -1);
+  int64_t entries = 0;
+  for (int bh = 0; bh < BH; ++bh)
+    for (int qt = 0; qt < n_qt; ++qt) {
+      const int64_t t = int64_t(bh) * n_qt + qt;
+      const int I0 = qt * qpt;
+      const int nq = std::min(qpt, n - I0);
+      for (int q = 0; q < nq; ++q) {
+        const int64_t r = int64_t(bh) * n + I0 + q;
+        for (int64_t e = row_ptr[r]; e < row_ptr[r + 1]; ++e)
+          if (stamp[col_idx[e]] != t) {
+            stamp[col_idx[e]] = t;
+            ++entries;
+          }
+      }
+    }
+  return entries;
 }
 
 // bf16 views of fp32 inputs, converted on the stream into temporaries.
@@ -198,6 +244,21 @@ int losa_pattern_export(const losa_pattern* p, int32_t* row_ptr, int32_t* col_id
       return LOSA_ERR_CUDA;
   }
   return cudaStreamSynchronize(s) == cudaSuccess ? LOSA_OK : LOSA_ERR_CUDA;
+}
+
+int losa_pattern_import(const int32_t* row_ptr, const int32_t* col_idx,
+                        const int64_t* retained_fx, const int64_t* total_fx, int B, int H,
+                        int n_blocks, int block, losa_pattern** out, void* stream) {
+  if (out) *out = nullptr;
+  if (!row_ptr || !col_idx || !out) return LOSA_ERR_ARG;
+  if (B < 1 || H < 1 || n_blocks < 1 || n_blocks > 2047) return LOSA_ERR_ARG;
+  if (block != 32 && block != 64 && block != 128) return LOSA_ERR_ARG;
+  if (int64_t(B) * H > 65535) return LOSA_ERR_ARG;
+  const int64_t tile_entries = validate_csr(row_ptr, col_idx, B * H, n_blocks, block);
+  if (tile_entries < 0) return LOSA_ERR_ARG;
+  if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
+  return import_pattern(row_ptr, col_idx, retained_fx, total_fx, B, H, n_blocks, block,
+                        tile_entries, out, static_cast<cudaStream_t>(stream));
 }
 
 int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, int d, int L,

@@ -64,4 +64,12 @@ cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStrea
 int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
                   losa_pattern** out, cudaStream_t stream);
 
+// Builds a pattern from a host CSR that the caller has validated (row_ptr
+// monotone from 0 with non-empty rows, columns strictly ascending in
+// [0, n)); tile_entries is the total of the 128-row tiles' union sizes.
+// Returns a losa_status.
+int import_pattern(const int32_t* row_ptr, const int32_t* col_idx, const int64_t* retained_fx,
+                   const int64_t* total_fx, int B, int H, int n, int block,
+                   int64_t tile_entries, losa_pattern** out, cudaStream_t stream);
+
 }  // namespace losa

@@ -267,6 +267,56 @@ __global__ void order_scatter_kernel(const int* __restrict__ tile_count, int T, 
     order[atomicAdd(&cursor[order_key(t, n_qt, n, tile_count)], 1)] = t;
 }
 
+// Union entries of one 128-row query tile from the CSR rows of its query
+// blocks, for a pattern that is imported rather than selected. kWrite =
+// false counts the tile's entries into tile_count; kWrite = true writes them
+// (J | mask << 16, ascending J) at tile_ptr. The host has checked that every
+// row's columns are strictly ascending and lie in [0, n), so within one row
+// no two threads touch the same byte of `masks`.
+template <bool kWrite>
+__global__ void __launch_bounds__(kSelThreads)
+    csr_tile_kernel(const int* __restrict__ row_ptr, const int* __restrict__ col_idx, int n,
+                    int qpt, int n_qt, int* __restrict__ tile_count,
+                    const int* __restrict__ tile_ptr, int* __restrict__ tile_entry) {
+  using Reduce = cub::BlockReduce<int, kSelThreads>;
+  using Scan = cub::BlockScan<int, kSelThreads>;
+  __shared__ union {
+    typename Reduce::TempStorage reduce;
+    typename Scan::TempStorage scan;
+  } tmp;
+  __shared__ unsigned char masks[2048];
+  const int t = blockIdx.x;
+  const int bh = t / n_qt, qt = t % n_qt;
+  const int I0 = qt * qpt;
+  const int nq = min(qpt, n - I0);
+  const int row0 = bh * n + I0;
+  for (int J = threadIdx.x; J < n; J += kSelThreads) masks[J] = 0;
+  __syncthreads();
+  for (int q = 0; q < nq; ++q) {
+    const int e1 = row_ptr[row0 + q + 1];
+    for (int e = row_ptr[row0 + q] + threadIdx.x; e < e1; e += kSelThreads)
+      masks[col_idx[e]] |= (unsigned char)(1u << q);
+    __syncthreads();
+  }
+  if (!kWrite) {
+    int c = 0;
+    for (int J = threadIdx.x; J < n; J += kSelThreads) c += masks[J] != 0;
+    const int total = Reduce(tmp.reduce).Sum(c);
+    if (threadIdx.x == 0) tile_count[t] = total;
+    return;
+  }
+  int base = tile_ptr[t];
+  for (int c0 = 0; c0 < n; c0 += kSelThreads) {
+    const int J = c0 + threadIdx.x;
+    const unsigned m = (J < n) ? masks[J] : 0u;
+    int ex, tot;
+    Scan(tmp.scan).ExclusiveSum(int(m != 0), ex, tot);
+    __syncthreads();
+    if (m) tile_entry[base + ex] = J | int(m << 16);
+    base += tot;
+  }
+}
+
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
@@ -374,6 +424,102 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
     return fail(LOSA_ERR_CUDA);
   }
   cudaFreeAsync(scratch, stream);
+  *out = p;
+  return LOSA_OK;
+}
+
+int import_pattern(const int32_t* row_ptr, const int32_t* col_idx, const int64_t* retained_fx,
+                   const int64_t* total_fx, int B, int H, int n, int block,
+                   int64_t tile_entries, losa_pattern** out, cudaStream_t stream) {
+  const int BH = B * H;
+  const int64_t R = int64_t(BH) * n;
+  const int L_pad = n * block;
+  const int n_qt = (L_pad + 127) / 128;
+  const int qpt = 128 / block;
+  const int64_t T = int64_t(BH) * n_qt;
+  const int64_t nnz = row_ptr[R];
+
+  losa_pattern* p = new losa_pattern{};
+  p->B = B;
+  p->H = H;
+  p->n_blocks = n;
+  p->block = block;
+  p->n_qt = n_qt;
+  p->n_tiles = T;
+  p->nnz = nnz;
+  p->tile_entries = tile_entries;
+  p->stream = stream;
+  cudaGetDevice(&p->device);
+
+  // Same arrays and layout as a selected pattern.
+  const size_t o_row = 0;
+  const size_t o_tptr = o_row + align256((R + 1) * 4);
+  const size_t o_tord = o_tptr + align256((T + 1) * 4);
+  const size_t o_ret = o_tord + align256(T * 4);
+  const size_t o_tot = o_ret + align256(R * 8);
+  const size_t fixed_bytes = o_tot + align256(R * 8);
+  const size_t list_bytes = align256(size_t(nnz) * 4) + align256(size_t(tile_entries) * 4);
+  const int64_t n_keys = int64_t(BH) * (n + 1);
+  const size_t s_tcnt = 0;
+  const size_t s_hist = s_tcnt + align256(T * 4);
+  const size_t s_cur = s_hist + align256(n_keys * 4);
+  const size_t scratch_bytes = s_cur + align256((n_keys + 1) * 4);
+
+  char* fixed = static_cast<char*>(pool_alloc(fixed_bytes, stream));
+  char* lists = static_cast<char*>(pool_alloc(list_bytes, stream));
+  char* scratch = static_cast<char*>(pool_alloc(scratch_bytes, stream));
+  auto fail = [&](int code) {
+    if (fixed) cudaFreeAsync(fixed, stream);
+    if (lists) cudaFreeAsync(lists, stream);
+    if (scratch) cudaFreeAsync(scratch, stream);
+    cudaStreamSynchronize(stream);
+    delete p;
+    return code;
+  };
+  if (!fixed || !lists || !scratch) return fail(LOSA_ERR_NOMEM);
+  p->row_ptr = reinterpret_cast<int32_t*>(fixed + o_row);
+  p->tile_ptr = reinterpret_cast<int32_t*>(fixed + o_tptr);
+  p->tile_order = reinterpret_cast<int32_t*>(fixed + o_tord);
+  p->retained_fx = reinterpret_cast<int64_t*>(fixed + o_ret);
+  p->total_fx = reinterpret_cast<int64_t*>(fixed + o_tot);
+  p->col_idx = reinterpret_cast<int32_t*>(lists);
+  p->tile_entry = reinterpret_cast<int32_t*>(lists + align256(size_t(nnz) * 4));
+  auto* tcnt = reinterpret_cast<int*>(scratch + s_tcnt);
+  auto* hist = reinterpret_cast<int*>(scratch + s_hist);
+  auto* cursor = reinterpret_cast<int*>(scratch + s_cur);
+
+  bool ok = cudaMemcpyAsync(p->row_ptr, row_ptr, size_t(R + 1) * 4, cudaMemcpyHostToDevice,
+                            stream) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(p->col_idx, col_idx, size_t(nnz) * 4, cudaMemcpyHostToDevice,
+                             stream) == cudaSuccess;
+  // Fixed-point sums are carried over when given, else marked unknown (-1).
+  ok = ok && (retained_fx ? cudaMemcpyAsync(p->retained_fx, retained_fx, size_t(R) * 8,
+                                            cudaMemcpyHostToDevice, stream)
+                          : cudaMemsetAsync(p->retained_fx, 0xff, size_t(R) * 8, stream)) ==
+                 cudaSuccess;
+  ok = ok && (total_fx ? cudaMemcpyAsync(p->total_fx, total_fx, size_t(R) * 8,
+                                         cudaMemcpyHostToDevice, stream)
+                       : cudaMemsetAsync(p->total_fx, 0xff, size_t(R) * 8, stream)) ==
+                 cudaSuccess;
+  if (!ok) return fail(LOSA_ERR_CUDA);
+
+  csr_tile_kernel<false><<<unsigned(T), kSelThreads, 0, stream>>>(
+      p->row_ptr, p->col_idx, n, qpt, n_qt, tcnt, nullptr, nullptr);
+  scan_kernel<<<1, 1024, 0, stream>>>(tcnt, int(T), p->tile_ptr);
+  csr_tile_kernel<true><<<unsigned(T), kSelThreads, 0, stream>>>(
+      p->row_ptr, p->col_idx, n, qpt, n_qt, nullptr, p->tile_ptr, p->tile_entry);
+  cudaMemsetAsync(hist, 0, n_keys * sizeof(int), stream);
+  const int og = int(std::min<int64_t>((T + 255) / 256, 1024));
+  order_hist_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n_qt, n, hist);
+  scan_kernel<<<1, 1024, 0, stream>>>(hist, int(n_keys), cursor);
+  order_scatter_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n_qt, n, cursor, p->tile_order);
+  if (cudaGetLastError() != cudaSuccess) return fail(LOSA_ERR_CUDA);
+  cudaFreeAsync(scratch, stream);
+  scratch = nullptr;
+  // The caller may release its host arrays (pinned ones included) on return.
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return fail(LOSA_ERR_CUDA);
+  p->fixed_mem = fixed;
+  p->list_mem = lists;
   *out = p;
   return LOSA_OK;
 }

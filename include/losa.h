@@ -159,6 +159,35 @@ int losa_pattern_export(const losa_pattern* p, int32_t* row_ptr, int32_t* col_id
                         int32_t* tile_entry, int32_t* tile_order, void* stream);
 
 /*
+ * losa_pattern_import - rebuilds a pattern from a stored CSR, the inverse of
+ * losa_pattern_export (ubos.tech LoSA post, Phase 2: the mask "is stored
+ * for reuse"), so a frozen pattern can outlive the process that selected it
+ * or come from elsewhere.
+ *
+ *   row_ptr      [B*H*n_blocks + 1] int32, HOST memory; row r = (b*H + h)*n
+ *                + I lists query block I's kept key blocks.
+ *   col_idx      [row_ptr[last]] int32, HOST memory.
+ *   retained_fx, total_fx
+ *                [B*H*n_blocks] int64 HOST memory or NULL; copied into the
+ *                pattern as given, or set to -1 (unknown) when NULL.
+ *   out          receives a new pattern on LOSA_OK, else NULL.
+ *
+ *   The CSR is checked on the host before any device work: row_ptr[0] = 0,
+ *   every row holds 1..n_blocks entries, and each row's columns are strictly
+ *   ascending in [0, n_blocks) (as losa_select writes them). The sparse
+ *   kernel's tile lists are then rebuilt on the device from the CSR; a
+ *   pattern exported from losa_select and imported again gives the same
+ *   row_ptr, col_idx, tile_ptr and tile_entry, and tile_order up to the order
+ *   of tiles with equal keys. The host arrays are read before the call
+ *   returns (it synchronises `stream`) and stay the caller's.
+ *   Returns LOSA_ERR_ARG (null pointer, sizes as for losa_select, an invalid
+ *   CSR), LOSA_ERR_NOMEM, LOSA_ERR_CUDA, LOSA_ERR_UNSUPPORTED.
+ */
+int losa_pattern_import(const int32_t* row_ptr, const int32_t* col_idx,
+                        const int64_t* retained_fx, const int64_t* total_fx, int B, int H,
+                        int n_blocks, int block, losa_pattern** out, void* stream);
+
+/*
  * losa_sparse_attn - later steps: attention of fresh Q/K/V restricted to the
  * frozen retained key blocks (Phase 3 - Repeated Sparse Inference, ubos.tech
  * LoSA post; legiblepapers.com "Summary & Methodology Analysis").

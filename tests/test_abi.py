@@ -101,3 +101,51 @@ def test_null_handles(losa):
     assert lib.losa_sparse_attn(FAKE, FAKE, FAKE, 0, 64, 10, 0.1, None, FAKE, 1, None, None) == -1
     assert lib.losa_pattern_export(None, None, None, None, None, None, None, None, None) == -1
     lib.losa_free(None)  # no-op
+
+
+def _import(losa, row_ptr, col_idx, B=1, H=1, n=4, block=64):
+    rp = (ctypes.c_int32 * len(row_ptr))(*row_ptr)
+    ci = (ctypes.c_int32 * max(len(col_idx), 1))(*col_idx)
+    out = ctypes.c_void_p(1)
+    st = losa.lib().losa_pattern_import(rp, ci, None, None, B, H, n, block, ctypes.byref(out),
+                                        None)
+    assert out.value is None  # *out is cleared on every failure
+    return st
+
+
+# One head, n = 4 key blocks, so 4 CSR rows; each case breaks one rule.
+@pytest.mark.parametrize("row_ptr,col_idx", [
+    ([1, 2, 3, 4, 5], [0, 0, 0, 0, 0]),            # row_ptr[0] != 0
+    ([0, 1, 1, 2, 3], [0, 1, 2]),                  # an empty row
+    ([0, 5, 6, 7, 8], [0, 1, 2, 3, 3, 0, 0, 0]),   # a row longer than n
+    ([0, 2, 3, 4, 5], [1, 0, 0, 0, 0]),            # columns not ascending
+    ([0, 2, 3, 4, 5], [1, 1, 0, 0, 0]),            # a repeated column
+    ([0, 1, 2, 3, 4], [0, 4, 0, 0]),               # a column >= n
+    ([0, 1, 2, 3, 4], [0, -1, 0, 0]),              # a negative column
+    ([0, 1, 2, 1, 4], [0, 1, 2, 3]),               # row_ptr decreasing
+])
+def test_pattern_import_rejects_invalid_csr(losa, row_ptr, col_idx):
+    assert _import(losa, row_ptr, col_idx) == -1
+
+
+def test_pattern_import_rejects_bad_shapes_and_nulls(losa):
+    lib = losa.lib()
+    out = ctypes.c_void_p()
+    rp = (ctypes.c_int32 * 5)(0, 1, 2, 3, 4)
+    ci = (ctypes.c_int32 * 4)(0, 1, 2, 3)
+    assert lib.losa_pattern_import(None, ci, None, None, 1, 1, 4, 64, ctypes.byref(out), None) == -1
+    assert lib.losa_pattern_import(rp, None, None, None, 1, 1, 4, 64, ctypes.byref(out), None) == -1
+    assert lib.losa_pattern_import(rp, ci, None, None, 1, 1, 4, 64, None, None) == -1
+    assert lib.losa_pattern_import(rp, ci, None, None, 1, 1, 4, 48, ctypes.byref(out), None) == -1
+    assert lib.losa_pattern_import(rp, ci, None, None, 1, 1, 2048, 64, ctypes.byref(out),
+                                   None) == -1
+    assert lib.losa_pattern_import(rp, ci, None, None, 0, 1, 4, 64, ctypes.byref(out), None) == -1
+
+
+def test_pattern_import_accepts_a_valid_csr_up_to_the_device_check(losa):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("device path covered by the GPU tests")
+    # Valid (diagonal plus one neighbour): passes the host checks, then the
+    # device check reports that no sm_100 GPU is present.
+    assert _import(losa, [0, 2, 4, 6, 7], [0, 1, 0, 1, 2, 3, 3]) == -6
