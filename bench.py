@@ -79,11 +79,16 @@ def load_peaks():
 
 
 def attention_source_sha():
+    """Hash of the attention kernel's code: the two sources with // comments,
+    trailing blanks and empty lines removed (a comment edit keeps the hash)."""
     import hashlib
     h = hashlib.sha256()
     for f in ("losa_attention.cuh", "losa_device.cuh"):
-        with open(os.path.join(ROOT, "block_sparse_attention_losa_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "block_sparse_attention_losa_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

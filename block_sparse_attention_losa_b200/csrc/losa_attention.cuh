@@ -8,8 +8,8 @@
 //   warp 9     MMA issuer (one thread) and TMEM owner,
 //   warps 10-11 idle.
 // The kernel launches with 168 registers per thread (384 x 168 = 64,512);
-// the third warpgroup gives registers back (setmaxnreg to 40) and the two
-// softmax warpgroups take them (to 232): 2*128*232 + 128*40 = 64,512.
+// the third warpgroup gives registers back (setmaxnreg to 72) and the two
+// softmax warpgroups take them (to 216): 2*128*216 + 128*72 = 64,512.
 // TMEM (512 columns): S_t at columns [128 t, 128 t + BN), O_t at 256 + t D.
 // Per key tile j of tile t: S_t = Q_t K_j^T (tcgen05 kind::f16, bf16 operands
 // from 128B-swizzled smem, fp32 in TMEM); the softmax warps read S_t, write
@@ -504,25 +504,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const float mx2 = mx * sl2;
 
-      // Raise the max (and rescale O_t in TMEM) whenever this tile exceeds
-      // it. S_t(j) completing implies PV_t(j-1) completed, so O_t is at rest.
+      // Raise the max whenever this tile exceeds it; O_t is rescaled to
+      // match after the exponentials below.
       float alpha = 1.f;
       if (mx2 > m_used) {
         if (m_used != NEG_INF) alpha = ex2_approx(m_used - mx2);
         m_used = mx2;
       }
-      if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
+      const bool rescale = __any_sync(0xffffffffu, alpha != 1.f) && j > 0;
+      if (rescale) {
         l *= alpha;
         l_c *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(o_col + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(o_col + c * 32, o);
-        }
       }
       const float msub = (m_used == NEG_INF) ? 0.f : m_used;
       // Exponent offset per entry: -msub, or -inf for an entry this row's
@@ -557,6 +549,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         tmem_st16(s_col + c * 16, pk);
+      }
+      if (rescale) {
+        // O_t *= alpha. S_t(j) completing implies PV_t(j-1) completed, so
+        // O_t is at rest; S's registers are free by now, so all of O's
+        // columns make one TMEM round trip instead of one per 32 columns.
+        float o[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tmem_ld32(o_col + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
+        tmem_ld_wait();
+        const f32x2 a2 = f2_make(alpha, alpha);
+#pragma unroll
+        for (int e = 0; e < D; e += 2) f2_split(f2_mul(f2_make(o[e], o[e + 1]), a2), o[e], o[e + 1]);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tmem_st32(o_col + c * 32, *reinterpret_cast<const float(*)[32]>(&o[c * 32]));
       }
       const float tsum = f2_sum(ts2[0]) + f2_sum(ts2[1]);
       {  // Kahan: l += tsum
