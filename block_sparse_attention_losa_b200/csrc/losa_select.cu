@@ -50,90 +50,131 @@ __device__ __forceinline__ bool reaches(unsigned long long C, unsigned long long
   return ((unsigned __int128)C << 48) >= (unsigned __int128)tau_fx * S;
 }
 
-// One CTA per row: the cut key, kept count, kept and total fixed-point mass.
-// The row's sort keys are sorted ascending in shared memory with a bitonic
-// network (NP = n rounded up to a power of two, padded with keys that sort
-// last), the fixed-point masses are prefix-summed in that order, and the cut
-// is the first position k where 2^48 * C_k >= tau_fx * S (exact, 128-bit).
-// No atomics, so the result does not depend on scheduling.
-template <int NP>
-__global__ void __launch_bounds__(kSelThreads)
-    select_cut_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
-                      unsigned long long* __restrict__ cut_key, int* __restrict__ count,
-                      long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
-                      int* status) {
-  constexpr int IPT = NP / kSelThreads > 0 ? NP / kSelThreads : 1;  // keys per thread
-  constexpr int NT = NP / IPT;                                       // threads holding keys
-  using Scan = cub::BlockScan<unsigned long long, kSelThreads>;
-  using Reduce = cub::BlockReduce<int, kSelThreads>;
-  __shared__ unsigned long long keys[NP];
-  __shared__ typename Scan::TempStorage scan_tmp;
-  __shared__ typename Reduce::TempStorage red_tmp;
-  __shared__ int sh_bad, sh_k;
+// One warp per row: the cut key, kept count, kept and total fixed-point
+// mass. The row's NP sort keys (n rounded up to a power of two, padded with
+// keys that sort last) live in registers, IPT = NP / 32 per lane, element
+// i = lane * IPT + r. A bitonic network sorts them ascending: exchanges
+// whose partner sits in the same lane (stride < IPT) stay in registers, the
+// others (stride >= IPT) go through warp shuffles. The fixed-point masses
+// are then prefix-summed in sorted order and the cut is the first position
+// k where 2^48 * C_k >= tau_fx * S (exact, 128-bit). No atomics and no
+// shared memory, so the result does not depend on scheduling.
+constexpr int kCutWarps = 4;  // rows per CTA
 
-  const int row = blockIdx.x;
+__device__ __forceinline__ unsigned long long umin64(unsigned long long a, unsigned long long b) {
+  return a < b ? a : b;
+}
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
+  return a < b ? b : a;
+}
+
+// Exchanges between elements r and r + stride of this lane (stride < IPT).
+template <int IPT, int STRIDE>
+__device__ __forceinline__ void bitonic_in_lane(unsigned long long (&k)[IPT], int lane, int size) {
+#pragma unroll
+  for (int r = 0; r < IPT; ++r) {
+    if ((r & STRIDE) == 0) {
+      const bool up = ((lane * IPT + r) & size) == 0;
+      const unsigned long long a = k[r], b = k[r + STRIDE];
+      k[r] = up ? umin64(a, b) : umax64(a, b);
+      k[r + STRIDE] = up ? umax64(a, b) : umin64(a, b);
+    }
+  }
+  if constexpr (STRIDE > 1) bitonic_in_lane<IPT, STRIDE / 2>(k, lane, size);
+}
+
+// The in-lane part of one merge step of `size`: strides min(size / 2, S0)
+// down to 1.
+template <int IPT, int S0>
+__device__ __forceinline__ void bitonic_in_lane_from(unsigned long long (&k)[IPT], int lane,
+                                                     int size) {
+  if constexpr (S0 >= 1) {
+    if (size / 2 >= S0)
+      bitonic_in_lane<IPT, S0>(k, lane, size);
+    else
+      bitonic_in_lane_from<IPT, S0 / 2>(k, lane, size);
+  }
+}
+
+template <int NP>
+__global__ void __launch_bounds__(32 * kCutWarps)
+    select_cut_kernel(const float* __restrict__ mass, int64_t R, int n,
+                      unsigned long long tau_fx, unsigned long long* __restrict__ cut_key,
+                      int* __restrict__ count, long long* __restrict__ retained_fx,
+                      long long* __restrict__ total_fx, int* status) {
+  constexpr int IPT = NP / 32;
+  static_assert(IPT >= 2 && (IPT & (IPT - 1)) == 0, "NP must be a power of two >= 64");
+  const int lane = threadIdx.x & 31;
+  const int64_t row = int64_t(blockIdx.x) * kCutWarps + (threadIdx.x >> 5);
+  if (row >= R) return;  // whole warps only
   const float* mrow = mass + size_t(row) * n;
-  if (threadIdx.x == 0) sh_bad = 0;
-  __syncthreads();
+
+  unsigned long long k[IPT];
   bool bad = false;
-  for (int J = threadIdx.x; J < NP; J += kSelThreads) {
+#pragma unroll
+  for (int r = 0; r < IPT; ++r) {
+    const int J = lane * IPT + r;
     unsigned long long key = kNoKey;
     if (J < n) {
       long long x;
       bad |= !to_fixed(mrow[J], x);
       key = sort_key(x, J);
     }
-    keys[J] = key;
+    k[r] = key;
   }
-  if (bad) sh_bad = 1;
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(status, kStatusOk, kStatusBadMass);
+
   // Bitonic sort, ascending.
   for (int size = 2; size <= NP; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int pr = threadIdx.x; pr < NP / 2; pr += kSelThreads) {
-        const int i = 2 * stride * (pr / stride) + (pr % stride);
-        const int k = i + stride;
-        const unsigned long long a = keys[i], b = keys[k];
-        const bool up = (i & size) == 0;
-        if ((a > b) == up) {
-          keys[i] = b;
-          keys[k] = a;
-        }
+    for (int stride = size >> 1; stride >= IPT; stride >>= 1) {
+      const int lx = stride / IPT;  // partner lane = lane ^ lx
+      const bool up = ((lane * IPT) & size) == 0;
+      const bool lower = (lane & lx) == 0;
+#pragma unroll
+      for (int r = 0; r < IPT; ++r) {
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, k[r], lx);
+        k[r] = (lower == up) ? umin64(k[r], o) : umax64(k[r], o);
       }
     }
+    bitonic_in_lane_from<IPT, IPT / 2>(k, lane, size);
   }
-  __syncthreads();
-  // Fixed-point masses in sorted order (thread t owns positions
-  // [t*IPT, t*IPT + IPT)); padding keys carry no mass.
-  unsigned long long xs[IPT];
+
+  // Fixed-point masses in sorted order; padding keys carry no mass.
+  auto xval = [](unsigned long long key) -> unsigned long long {
+    return key == kNoKey ? 0ull : kXMax - (key >> 11);
+  };
+  unsigned long long T = 0;
 #pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    const int pos = threadIdx.x * IPT + i;
-    const unsigned long long key = (threadIdx.x < NT) ? keys[pos] : kNoKey;
-    xs[i] = (key == kNoKey) ? 0ull : kXMax - (key >> 11);
+  for (int r = 0; r < IPT; ++r) T += xval(k[r]);
+  unsigned long long incl = T;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
   }
-  unsigned long long incl[IPT], S;
-  Scan(scan_tmp).InclusiveSum(xs, incl, S);
+  const unsigned long long S = __shfl_sync(0xffffffffu, incl, 31);
   // First position whose running sum reaches the threshold (k >= 1; the full
   // row always reaches it, and an all-zero row stops at its first key).
-  int first = NP;
+  unsigned long long C = incl - T;
+  unsigned first = unsigned(NP);
+  unsigned long long key_at = 0, c_at = 0;
 #pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    const int pos = threadIdx.x * IPT + i;
-    if (threadIdx.x < NT && pos < n && first == NP && reaches(incl[i], tau_fx, S)) first = pos;
+  for (int r = 0; r < IPT; ++r) {
+    C += xval(k[r]);
+    const int pos = lane * IPT + r;
+    if (first == unsigned(NP) && pos < n && reaches(C, tau_fx, S)) {
+      first = unsigned(pos);
+      key_at = k[r];
+      c_at = C;
+    }
   }
-  const int kmin = Reduce(red_tmp).Reduce(first, cub::Min());
-  if (threadIdx.x == 0) sh_k = kmin;
-  __syncthreads();
-  const int kcut = sh_k;
-  if (threadIdx.x < NT && kcut / IPT == int(threadIdx.x)) {
-    // The thread holding the cut position writes the row's results.
-    const int i = kcut % IPT;
-    cut_key[row] = keys[kcut];
-    count[row] = kcut + 1;
-    retained_fx[row] = (long long)incl[i];
+  const unsigned kcut = __reduce_min_sync(0xffffffffu, first);
+  if (first == kcut && kcut < unsigned(NP)) {
+    // The lane holding the cut position writes the row's results.
+    cut_key[row] = key_at;
+    count[row] = int(kcut) + 1;
+    retained_fx[row] = (long long)c_at;
     total_fx[row] = (long long)S;
-    if (sh_bad) atomicCAS(status, kStatusOk, kStatusBadMass);
   }
 }
 
@@ -141,13 +182,16 @@ __global__ void __launch_bounds__(kSelThreads)
 cudaError_t launch_select_cut(const float* mass, int64_t R, int n, unsigned long long tau_fx,
                               unsigned long long* cut, int* cnt, long long* retained,
                               long long* total, int* status, cudaStream_t stream) {
-#define LOSA_CUT(NP_)                                                                      \
-  if (n <= NP_) {                                                                          \
-    select_cut_kernel<NP_><<<unsigned(R), kSelThreads, 0, stream>>>(mass, n, tau_fx, cut, \
-                                                                     cnt, retained, total, \
-                                                                     status);              \
-    return cudaGetLastError();                                                             \
+  const unsigned grid = unsigned((R + kCutWarps - 1) / kCutWarps);
+#define LOSA_CUT(NP_)                                                                   \
+  if (n <= NP_) {                                                                       \
+    select_cut_kernel<NP_><<<grid, 32 * kCutWarps, 0, stream>>>(mass, R, n, tau_fx, cut, \
+                                                                 cnt, retained, total,   \
+                                                                 status);                \
+    return cudaGetLastError();                                                          \
   }
+  LOSA_CUT(64)
+  LOSA_CUT(128)
   LOSA_CUT(256)
   LOSA_CUT(512)
   LOSA_CUT(1024)
