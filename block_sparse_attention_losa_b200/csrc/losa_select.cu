@@ -178,6 +178,122 @@ __global__ void __launch_bounds__(32 * kCutWarps)
   }
 }
 
+// The same cut for rows of NP >= 1024 keys, where one warp would need 64
+// keys per lane: one CTA of WPR warps per row, IPT = NP / (32 WPR) keys per
+// thread (element i = t * IPT + r, t = thread of the CTA). Exchanges within a
+// thread stay in registers, within a warp go through shuffles, and across
+// warps (stride >= 32 IPT) through shared memory.
+template <int NP, int WPR>
+__global__ void __launch_bounds__(32 * WPR)
+    select_cut_cta_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
+                          unsigned long long* __restrict__ cut_key, int* __restrict__ count,
+                          long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
+                          int* status) {
+  constexpr int NT = 32 * WPR;
+  constexpr int IPT = NP / NT;
+  static_assert(IPT >= 2 && (IPT & (IPT - 1)) == 0, "NP / (32 WPR) must be a power of two >= 2");
+  __shared__ unsigned long long xk[NP];  // cross-warp exchange, xk[r * NT + t]
+  __shared__ unsigned long long wsum[WPR];
+  __shared__ unsigned wmin[WPR];
+  const int t = threadIdx.x;
+  const int lane = t & 31, w = t >> 5;
+  const int64_t row = blockIdx.x;
+  const float* mrow = mass + size_t(row) * n;
+
+  unsigned long long k[IPT];
+  bool bad = false;
+#pragma unroll
+  for (int r = 0; r < IPT; ++r) {
+    const int J = t * IPT + r;
+    unsigned long long key = kNoKey;
+    if (J < n) {
+      long long x;
+      bad |= !to_fixed(mrow[J], x);
+      key = sort_key(x, J);
+    }
+    k[r] = key;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(status, kStatusOk, kStatusBadMass);
+
+  // Bitonic sort, ascending.
+  for (int size = 2; size <= NP; size <<= 1) {
+    const bool up = ((t * IPT) & size) == 0;  // same for all of this thread's elements
+    for (int stride = size >> 1; stride >= 32 * IPT; stride >>= 1) {
+      const int tx = stride / IPT;  // partner thread = t ^ tx, in another warp
+      const bool lower = (t & tx) == 0;
+#pragma unroll
+      for (int r = 0; r < IPT; ++r) xk[r * NT + t] = k[r];
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < IPT; ++r) {
+        const unsigned long long o = xk[r * NT + (t ^ tx)];
+        k[r] = (lower == up) ? umin64(k[r], o) : umax64(k[r], o);
+      }
+      __syncthreads();
+    }
+    for (int stride = min(size >> 1, 16 * IPT); stride >= IPT; stride >>= 1) {
+      const int lx = stride / IPT;  // partner lane = lane ^ lx
+      const bool lower = (lane & lx) == 0;
+#pragma unroll
+      for (int r = 0; r < IPT; ++r) {
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, k[r], lx);
+        k[r] = (lower == up) ? umin64(k[r], o) : umax64(k[r], o);
+      }
+    }
+    bitonic_in_lane_from<IPT, IPT / 2>(k, t, size);
+  }
+
+  // Fixed-point masses in sorted order; padding keys carry no mass.
+  auto xval = [](unsigned long long key) -> unsigned long long {
+    return key == kNoKey ? 0ull : kXMax - (key >> 11);
+  };
+  unsigned long long T = 0;
+#pragma unroll
+  for (int r = 0; r < IPT; ++r) T += xval(k[r]);
+  unsigned long long incl = T;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  unsigned long long base = 0, S = 0;
+#pragma unroll
+  for (int i = 0; i < WPR; ++i) {
+    if (i < w) base += wsum[i];
+    S += wsum[i];
+  }
+  // First position whose running sum reaches the threshold (k >= 1; the full
+  // row always reaches it, and an all-zero row stops at its first key).
+  unsigned long long C = base + incl - T;
+  unsigned first = unsigned(NP);
+  unsigned long long key_at = 0, c_at = 0;
+#pragma unroll
+  for (int r = 0; r < IPT; ++r) {
+    C += xval(k[r]);
+    const int pos = t * IPT + r;
+    if (first == unsigned(NP) && pos < n && reaches(C, tau_fx, S)) {
+      first = unsigned(pos);
+      key_at = k[r];
+      c_at = C;
+    }
+  }
+  const unsigned wm = __reduce_min_sync(0xffffffffu, first);
+  if (lane == 0) wmin[w] = wm;
+  __syncthreads();
+  unsigned kcut = unsigned(NP);
+#pragma unroll
+  for (int i = 0; i < WPR; ++i) kcut = min(kcut, wmin[i]);
+  if (first == kcut && kcut < unsigned(NP)) {
+    // The thread holding the cut position writes the row's results.
+    cut_key[row] = key_at;
+    count[row] = int(kcut) + 1;
+    retained_fx[row] = (long long)c_at;
+    total_fx[row] = (long long)S;
+  }
+}
+
 // Launches the cut kernel with the smallest power-of-two capacity >= n.
 cudaError_t launch_select_cut(const float* mass, int64_t R, int n, unsigned long long tau_fx,
                               unsigned long long* cut, int* cnt, long long* retained,
@@ -194,9 +310,17 @@ cudaError_t launch_select_cut(const float* mass, int64_t R, int n, unsigned long
   LOSA_CUT(128)
   LOSA_CUT(256)
   LOSA_CUT(512)
-  LOSA_CUT(1024)
-  LOSA_CUT(2048)
 #undef LOSA_CUT
+  if (n <= 1024) {
+    select_cut_cta_kernel<1024, 2><<<unsigned(R), 64, 0, stream>>>(mass, n, tau_fx, cut, cnt,
+                                                                   retained, total, status);
+    return cudaGetLastError();
+  }
+  if (n <= 2048) {
+    select_cut_cta_kernel<2048, 4><<<unsigned(R), 128, 0, stream>>>(mass, n, tau_fx, cut, cnt,
+                                                                    retained, total, status);
+    return cudaGetLastError();
+  }
   return cudaErrorInvalidValue;
 }
 
