@@ -271,6 +271,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_wait_drain(&q_full[1], 0);
         for (int i = (kc > NSK ? kc - NSK : 0); i < kc; ++i) mbar_wait_drain(&k_full[i % NSK], (i / NSK) & 1);
         for (int i = (vc > NSV ? vc - NSV : 0); i < vc; ++i) mbar_wait_drain(&v_full[i % NSV], (i / NSV) & 1);
+      } else {
+        // A tile slot with no work (the last CTA of an odd tile count):
+        // nobody else waits for its Q copy, so let it land before exit.
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (n_it[t] == 0) mbar_wait_drain(&q_full[t], 0);
       }
     }
   } else if (warp == 9) {
