@@ -34,17 +34,20 @@
  *   - Attention is bidirectional: softmax(scale * q k^T) over the valid keys.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *     stream-ordered and return without a host synchronisation, except
- *     losa_select (one synchronisation, to size the CSR) and
- *     losa_check_status.
+ *     losa_select (one synchronisation, to size the CSR),
+ *     losa_pattern_export / losa_pattern_import (they finish their copies
+ *     before returning) and losa_check_status.
  *   - Every call returns LOSA_OK (0) or a negative losa_status; it checks
  *     its arguments on the host before touching the device and then leaves
  *     outputs untouched on LOSA_ERR_ARG.
  *   - Supported: d in {64, 128}; block in {32, 64, 128}; n <= 2047;
  *     B*H <= 65535; an sm_100 device.
- *   - The library keeps no global state besides one device status word per
- *     device (set by a kernel that ran out of a bounded wait, or by a bad
- *     mass value) and its CUDA function handles. Calls on different streams
- *     are independent.
+ *   - The library keeps no global state besides, per device, one status
+ *     word (set by a kernel that ran out of a bounded wait, or by a bad mass
+ *     value), one stream-ordered memory pool (patterns and scratch), the
+ *     fixed scratch array of losa_select_noalloc, and its CUDA function
+ *     handles. Calls on different streams are independent, except that
+ *     overlapping losa_select_noalloc calls share that scratch array.
  */
 #ifndef LOSA_H_
 #define LOSA_H_
