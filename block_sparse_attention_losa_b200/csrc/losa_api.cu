@@ -268,6 +268,9 @@ int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, 
   if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LOSA_ERR_ARG;
   const int L_pad = p->n_blocks * p->block;
   if (!valid_attn_shape(p->B, p->H, L, L_pad, d, p->block)) return LOSA_ERR_ARG;
+  int dev = -1;
+  // The pattern's arrays live on the device that built it.
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return LOSA_ERR_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return LOSA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_ARG;
   if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;

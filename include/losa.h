@@ -201,7 +201,8 @@ int losa_pattern_import(const int32_t* row_ptr, const int32_t* col_idx,
  *             softmax renormalised over the retained keys R(I) only.
  *   lse       [B, H, L_pad] fp32, may be NULL: log-sum-exp over the retained keys.
  *   Returns LOSA_ERR_ARG for a null pointer, a bad dtype, d not in {64, 128},
- *   L < 1, L > L_pad or L_pad - L >= block.
+ *   L < 1, L > L_pad, L_pad - L >= block, or a current device other than the
+ *   one the pattern was built on.
  */
 int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, int d,
                      int L, float scale, const losa_pattern* p,
