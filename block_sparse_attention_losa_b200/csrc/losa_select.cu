@@ -178,119 +178,185 @@ __global__ void __launch_bounds__(32 * kCutWarps)
   }
 }
 
-// The same cut for rows of NP >= 1024 keys, where one warp would need 64
-// keys per lane: one CTA of WPR warps per row, IPT = NP / (32 WPR) keys per
-// thread (element i = t * IPT + r, t = thread of the CTA). Exchanges within a
-// thread stay in registers, within a warp go through shuffles, and across
-// warps (stride >= 32 IPT) through shared memory.
-template <int NP, int WPR>
-__global__ void __launch_bounds__(32 * WPR)
-    select_cut_cta_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
-                          unsigned long long* __restrict__ cut_key, int* __restrict__ count,
-                          long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
-                          int* status) {
-  constexpr int NT = 32 * WPR;
-  constexpr int IPT = NP / NT;
-  static_assert(IPT >= 2 && (IPT & (IPT - 1)) == 0, "NP / (32 WPR) must be a power of two >= 2");
-  __shared__ unsigned long long xk[NP];  // cross-warp exchange, xk[r * NT + t]
-  __shared__ unsigned long long wsum[WPR];
-  __shared__ unsigned wmin[WPR];
+// Rows of more than 512 key blocks: one CTA per row. The keys are bucketed
+// by the leading five bits of x (the highest set bit and the four below it: 16 buckets per
+// octave of mass, x = 0 in bucket 0), so every key of a higher bucket has a
+// larger x than every key of a lower one. The bucket in which the running sum
+// over buckets in descending order first reaches the threshold is found with
+// a block scan, and only that bucket's keys are sorted (bitonic, in shared
+// memory): the keys of the buckets above fill the first positions of the
+// sorted order whatever their own order, so the cut (position, key and
+// prefix sum) is the one the full sort-and-accumulate definition gives.
+// Bucket sums and counts are integer atomics: the result does not depend on
+// scheduling.
+constexpr int kBkThreads = 256;
+constexpr int kBkPerThread = 4;
+constexpr int kBuckets = 1 + 49 * 16;  // x < 2^49
+constexpr int kBkCap = 2048;           // n <= 2047 keys, padded to a power of two
+static_assert(kBkThreads * kBkPerThread >= kBuckets, "bucket scan coverage");
+
+__device__ __forceinline__ int x_bucket(unsigned long long x) {
+  if (x == 0) return 0;
+  const int h = 63 - __clzll((long long)x);
+  const int sub = h >= 4 ? int((x >> (h - 4)) & 15u) : int((x << (4 - h)) & 15u);
+  return 1 + h * 16 + sub;
+}
+
+__global__ void __launch_bounds__(kBkThreads)
+    select_cut_bucket_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
+                             unsigned long long* __restrict__ cut_key, int* __restrict__ count,
+                             long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
+                             int* status) {
+  using ScanU = cub::BlockScan<unsigned long long, kBkThreads>;
+  using ScanI = cub::BlockScan<int, kBkThreads>;
+  using Reduce = cub::BlockReduce<int, kBkThreads>;
+  __shared__ unsigned long long hsum[kBuckets];
+  __shared__ int hcnt[kBuckets];
+  __shared__ unsigned long long cand[kBkCap];
+  __shared__ union {
+    typename ScanU::TempStorage scan_u;
+    typename ScanI::TempStorage scan_i;
+    typename Reduce::TempStorage reduce;
+  } tmp;
+  __shared__ unsigned long long sh_A, sh_S;
+  __shared__ int sh_b, sh_above, sh_m, sh_k;
   const int t = threadIdx.x;
-  const int lane = t & 31, w = t >> 5;
   const int64_t row = blockIdx.x;
   const float* mrow = mass + size_t(row) * n;
 
-  unsigned long long k[IPT];
+  for (int i = t; i < kBuckets; i += kBkThreads) {
+    hsum[i] = 0;
+    hcnt[i] = 0;
+  }
+  if (t == 0) sh_m = 0;
+  __syncthreads();
   bool bad = false;
-#pragma unroll
-  for (int r = 0; r < IPT; ++r) {
-    const int J = t * IPT + r;
-    unsigned long long key = kNoKey;
-    if (J < n) {
-      long long x;
-      bad |= !to_fixed(mrow[J], x);
-      key = sort_key(x, J);
-    }
-    k[r] = key;
+  for (int J = t; J < n; J += kBkThreads) {
+    long long x;
+    bad |= !to_fixed(mrow[J], x);
+    const int b = x_bucket((unsigned long long)x);
+    atomicAdd(&hsum[b], (unsigned long long)x);
+    atomicAdd(&hcnt[b], 1);
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(status, kStatusOk, kStatusBadMass);
+  if (__any_sync(0xffffffffu, bad) && (t & 31) == 0) atomicCAS(status, kStatusOk, kStatusBadMass);
+  __syncthreads();
 
-  // Bitonic sort, ascending.
-  for (int size = 2; size <= NP; size <<= 1) {
-    const bool up = ((t * IPT) & size) == 0;  // same for all of this thread's elements
-    for (int stride = size >> 1; stride >= 32 * IPT; stride >>= 1) {
-      const int tx = stride / IPT;  // partner thread = t ^ tx, in another warp
-      const bool lower = (t & tx) == 0;
+  // Buckets in descending order: thread t owns reversed positions
+  // [t * 4, t * 4 + 4), i.e. buckets kBuckets - 1 - pos.
+  unsigned long long ls = 0;
+  int lc = 0;
 #pragma unroll
-      for (int r = 0; r < IPT; ++r) xk[r * NT + t] = k[r];
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < IPT; ++r) {
-        const unsigned long long o = xk[r * NT + (t ^ tx)];
-        k[r] = (lower == up) ? umin64(k[r], o) : umax64(k[r], o);
-      }
-      __syncthreads();
+  for (int i = 0; i < kBkPerThread; ++i) {
+    const int pos = t * kBkPerThread + i;
+    if (pos < kBuckets) {
+      ls += hsum[kBuckets - 1 - pos];
+      lc += hcnt[kBuckets - 1 - pos];
     }
-    for (int stride = min(size >> 1, 16 * IPT); stride >= IPT; stride >>= 1) {
-      const int lx = stride / IPT;  // partner lane = lane ^ lx
-      const bool lower = (lane & lx) == 0;
-#pragma unroll
-      for (int r = 0; r < IPT; ++r) {
-        const unsigned long long o = __shfl_xor_sync(0xffffffffu, k[r], lx);
-        k[r] = (lower == up) ? umin64(k[r], o) : umax64(k[r], o);
-      }
-    }
-    bitonic_in_lane_from<IPT, IPT / 2>(k, t, size);
   }
-
-  // Fixed-point masses in sorted order; padding keys carry no mass.
+  unsigned long long sum_before, S;
+  ScanU(tmp.scan_u).ExclusiveSum(ls, sum_before, S);
+  __syncthreads();
+  int cnt_before;
+  ScanI(tmp.scan_i).ExclusiveSum(lc, cnt_before);
+  __syncthreads();
+  // First bucket (in descending order) whose inclusive sum reaches the
+  // threshold; an all-zero row (S = 0) stops at its first key, in bucket 0.
+  int first = kBuckets;
+  unsigned long long A_at = 0;
+  int above_at = 0;
+  {
+    unsigned long long A = sum_before;
+    int above = cnt_before;
+#pragma unroll
+    for (int i = 0; i < kBkPerThread; ++i) {
+      const int pos = t * kBkPerThread + i;
+      if (pos >= kBuckets || first != kBuckets) break;
+      const int b = kBuckets - 1 - pos;
+      if (S > 0 ? reaches(A + hsum[b], tau_fx, S) : b == 0) {
+        first = pos;
+        A_at = A;
+        above_at = above;
+      }
+      A += hsum[b];
+      above += hcnt[b];
+    }
+  }
+  const int pmin = Reduce(tmp.reduce).Reduce(first, cub::Min());
+  if (t == 0) sh_k = pmin;
+  __syncthreads();
+  if (first == sh_k && first < kBuckets) {
+    sh_b = kBuckets - 1 - first;
+    sh_A = A_at;
+    sh_above = above_at;
+    sh_S = S;
+  }
+  __syncthreads();
+  const int bstar = sh_b;
+  // The boundary bucket's keys (the row is in L1 by now).
+  for (int J = t; J < n; J += kBkThreads) {
+    long long x;
+    to_fixed(mrow[J], x);
+    if (x_bucket((unsigned long long)x) == bstar) cand[atomicAdd(&sh_m, 1)] = sort_key(x, J);
+  }
+  __syncthreads();
+  const int m = sh_m;
+  int np = 2;
+  while (np < m) np <<= 1;
+  for (int i = m + t; i < np; i += kBkThreads) cand[i] = kNoKey;
+  // Bitonic sort of the bucket, ascending.
+  for (int size = 2; size <= np; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int pr = t; pr < np / 2; pr += kBkThreads) {
+        const int i = 2 * stride * (pr / stride) + (pr % stride);
+        const int k = i + stride;
+        const unsigned long long a = cand[i], b = cand[k];
+        const bool up = (i & size) == 0;
+        if ((a > b) == up) {
+          cand[i] = b;
+          cand[k] = a;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // Prefix sums over the sorted bucket, on top of the buckets above it:
+  // thread t owns positions [t * per, t * per + per).
+  const int per = (np + kBkThreads - 1) / kBkThreads;
   auto xval = [](unsigned long long key) -> unsigned long long {
     return key == kNoKey ? 0ull : kXMax - (key >> 11);
   };
-  unsigned long long T = 0;
-#pragma unroll
-  for (int r = 0; r < IPT; ++r) T += xval(k[r]);
-  unsigned long long incl = T;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
+  unsigned long long local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int pos = t * per + i;
+    if (pos < m) local += xval(cand[pos]);
   }
-  if (lane == 31) wsum[w] = incl;
+  unsigned long long before;
+  ScanU(tmp.scan_u).ExclusiveSum(local, before);
   __syncthreads();
-  unsigned long long base = 0, S = 0;
-#pragma unroll
-  for (int i = 0; i < WPR; ++i) {
-    if (i < w) base += wsum[i];
-    S += wsum[i];
-  }
-  // First position whose running sum reaches the threshold (k >= 1; the full
-  // row always reaches it, and an all-zero row stops at its first key).
-  unsigned long long C = base + incl - T;
-  unsigned first = unsigned(NP);
-  unsigned long long key_at = 0, c_at = 0;
-#pragma unroll
-  for (int r = 0; r < IPT; ++r) {
-    C += xval(k[r]);
-    const int pos = t * IPT + r;
-    if (first == unsigned(NP) && pos < n && reaches(C, tau_fx, S)) {
-      first = unsigned(pos);
-      key_at = k[r];
-      c_at = C;
+  const unsigned long long St = sh_S;
+  unsigned long long C = sh_A + before;
+  int firstk = kBkCap;
+  for (int i = 0; i < per; ++i) {
+    const int pos = t * per + i;
+    if (pos >= m) break;
+    C += xval(cand[pos]);
+    if (reaches(C, tau_fx, St)) {
+      firstk = pos;
+      break;
     }
   }
-  const unsigned wm = __reduce_min_sync(0xffffffffu, first);
-  if (lane == 0) wmin[w] = wm;
+  const int kmin = Reduce(tmp.reduce).Reduce(firstk, cub::Min());
+  if (t == 0) sh_k = kmin;
   __syncthreads();
-  unsigned kcut = unsigned(NP);
-#pragma unroll
-  for (int i = 0; i < WPR; ++i) kcut = min(kcut, wmin[i]);
-  if (first == kcut && kcut < unsigned(NP)) {
-    // The thread holding the cut position writes the row's results.
-    cut_key[row] = key_at;
-    count[row] = int(kcut) + 1;
-    retained_fx[row] = (long long)c_at;
-    total_fx[row] = (long long)S;
+  const int p = sh_k;
+  if (p < m && p >= t * per && p < t * per + per) {
+    // The thread that owns the cut position writes the row's results; its
+    // running sum C stopped exactly there.
+    cut_key[row] = cand[p];
+    count[row] = sh_above + p + 1;
+    retained_fx[row] = (long long)C;
+    total_fx[row] = (long long)St;
   }
 }
 
@@ -311,14 +377,9 @@ cudaError_t launch_select_cut(const float* mass, int64_t R, int n, unsigned long
   LOSA_CUT(256)
   LOSA_CUT(512)
 #undef LOSA_CUT
-  if (n <= 1024) {
-    select_cut_cta_kernel<1024, 2><<<unsigned(R), 64, 0, stream>>>(mass, n, tau_fx, cut, cnt,
-                                                                   retained, total, status);
-    return cudaGetLastError();
-  }
-  if (n <= 2048) {
-    select_cut_cta_kernel<2048, 4><<<unsigned(R), 128, 0, stream>>>(mass, n, tau_fx, cut, cnt,
-                                                                    retained, total, status);
+  if (n < kBkCap) {
+    select_cut_bucket_kernel<<<unsigned(R), kBkThreads, 0, stream>>>(mass, n, tau_fx, cut, cnt,
+                                                                     retained, total, status);
     return cudaGetLastError();
   }
   return cudaErrorInvalidValue;
