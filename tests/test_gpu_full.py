@@ -15,6 +15,7 @@ from test_gpu_parity import LSE_ATOL, MASS_ATOL, O_MAX
 pytestmark = pytest.mark.gpu
 
 PER_HEAD = 2  # sampled query blocks per head
+SELECT_PER_HEAD = 16  # sampled rows per head for the selection-only check
 
 
 @pytest.fixture(scope="module")
@@ -58,6 +59,12 @@ def test_full_size_workload(losa, name):
     losa.check_status()
 
     mass_cpu = mass.cpu().numpy()
+    # Selection alone on a wider sample (it is cheap): bit-exact rows.
+    for (bb, h, I) in W.sample_query_blocks(wl, SELECT_PER_HEAD, seed=7):
+        r = (bb * wl.heads + h) * wl.n_blocks + I
+        kept, C, S = O.select_row(O.to_fixed(mass_cpu[bb, h, I]).tolist(), tau)
+        assert ex["col_idx"][rp[r]:rp[r + 1]].tolist() == kept
+        assert ret[r] == C and tot[r] == S
     for (bb, h, I) in W.sample_query_blocks(wl, PER_HEAD, seed=99):
         r = (bb * wl.heads + h) * wl.n_blocks + I
         # selection: bit-exact against the oracle on the GPU masses
