@@ -35,6 +35,8 @@ def test_reference_arm_two_ranks():
     assert len(lines) == 1, res.stdout
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["value"] > 0 and rec["steps"] == 2
+    assert rec["unit"] == "TFLOP/s" and rec["higher_is_better"] is True
+    assert rec["n_gpus"] == 2 and rec["warmup"] == 1 and rec["config"]["workload"] == "tiny"
     assert rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
 
