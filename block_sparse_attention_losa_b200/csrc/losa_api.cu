@@ -60,8 +60,6 @@ void* pool_alloc(size_t bytes, cudaStream_t stream) {
   return p;
 }
 
-namespace {
-
 bool is_sm100() {
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -70,6 +68,8 @@ bool is_sm100() {
     return false;
   return major == 10 && minor == 0;
 }
+
+namespace {
 
 bool valid_dtype(int dt) { return dt == LOSA_BF16 || dt == LOSA_FP32; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -319,6 +319,12 @@ int losa_selftest_wait(int64_t limit_cycles, void* stream) {
   return launch_wait_selftest(limit_cycles, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LOSA_OK
              : LOSA_ERR_CUDA;
+}
+
+int losa_set_wait_limit(int64_t limit_cycles) {
+  if (limit_cycles < 0 || limit_cycles > (int64_t(1) << 33)) return LOSA_ERR_ARG;
+  set_wait_limit(limit_cycles);
+  return LOSA_OK;
 }
 
 int losa_exp2_eval(const float* x, float* y, int64_t n, void* stream) {

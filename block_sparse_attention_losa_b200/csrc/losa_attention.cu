@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -11,6 +12,14 @@
 #include "losa_internal.h"
 
 namespace losa {
+
+// Wait limit of the attention kernels' mbarrier waits, in SM cycles.
+std::atomic<long long> g_wait_limit{kWaitLimitCycles};
+
+void set_wait_limit(long long cycles) {
+  g_wait_limit.store(cycles > 0 ? cycles : kWaitLimitCycles);
+}
+
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -144,6 +153,7 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, in
   p.mass = mass;
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
+  p.wait_limit = g_wait_limit.load();
   const dim3 grid((p.n_qt + 1) / 2, BH);  // two query tiles per CTA
 #define LOSA_DENSE_CASE(D_, NSK_, NSV_, BLK_)                                                   \
   if (d == D_ && block == BLK_)                                                                \
@@ -178,6 +188,7 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, in
   p.tile_order = pat->tile_order;
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
+  p.wait_limit = g_wait_limit.load();
   const int BH = pat->B * pat->H;
   p.n_tiles = int(pat->n_tiles);
   const dim3 grid(unsigned((pat->n_tiles + 1) / 2));  // two tiles per CTA

@@ -50,6 +50,7 @@ struct AttnParams {
   const int* tile_entry;  // sparse only
   const int* tile_order;  // sparse only
   int* status;
+  long long wait_limit;   // SM cycles a wait spins before it gives up
 };
 
 template <int D, int BN, int NSK, int NSV>
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const WaitCtx wc{abort_flag, p.status};
+  const WaitCtx wc{abort_flag, p.status, p.wait_limit};
 
   if (warp >= 8) {
   reg_dealloc<kControlRegs>();
@@ -524,7 +525,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const float msub = (m_used == NEG_INF) ? 0.f : m_used;
       // Exponent offset per entry: -msub, or -inf for an entry this row's
-      // query block does not keep (S is finite there, so exp2 gives 0).
+      // query block does not keep (S is finite there, so MUFU ex2 gives
+      // exactly 0; a column pair that took the FMA-pipe exp2 would give its
+      // clamped floor of ~2e-38 instead, see exp2_fma2).
       float nsub[EPI];
 #pragma unroll
       for (int e = 0; e < EPI; ++e) nsub[e] = on[e] ? -msub : NEG_INF;
@@ -653,8 +656,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int key0 = j * BN;
         // Padded query rows subtract +inf (their scores are finite: rows past
         // L hold finite values by contract, rows past L_pad read as zero), so
-        // they add exact zeros. Padded keys only occur in the last key tile,
-        // which takes its own warp-uniform branch.
+        // they add zeros: exact ones from MUFU ex2, and the FMA-pipe exp2's
+        // clamped floor (~2e-38 per entry, under 1e-33 per mass entry, far
+        // below fp32 resolution of any mass) in the columns that take it.
+        // Padded keys only occur in the last key tile, which takes its own
+        // warp-uniform branch.
         float part[NG];
         if (key0 + BN <= p.L) {
           const f32x2 sl2x2 = f2_make(sl2, sl2);

@@ -62,11 +62,13 @@ struct WaitCtx {
   long long limit = kWaitLimitCycles;  // SM cycles before a wait gives up
 };
 
+// The abort flag and the clock are checked after the first failed poll and
+// then every 64 polls, so a limit of a few cycles makes the first wait that
+// is not satisfied at once give up, whatever the polls' own latency.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t it = 0;; ++it) {
     if ((it & 63u) == 0) {
       if (*w.abort_flag) return false;
       if (clock64() - t0 > w.limit) {
@@ -75,6 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
         return false;
       }
     }
+    if (mbar_try_wait(bar, parity)) return true;
   }
 }
 

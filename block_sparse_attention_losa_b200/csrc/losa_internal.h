@@ -28,6 +28,9 @@ struct losa_pattern {
 
 namespace losa {
 
+// True when the current device is an sm_100 part (the only target built).
+bool is_sm100();
+
 // Device status word of the current device (lazily resolved per device).
 int* device_status_word();
 
@@ -49,6 +52,10 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, in
 cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, int L,
                           float scale, const losa_pattern* p, void* o, bool out_bf16,
                           float* lse, cudaStream_t stream);
+
+// Wait limit (SM cycles) of the attention kernels launched after the call;
+// 0 restores the default.
+void set_wait_limit(long long cycles);
 
 // One bounded mbarrier wait that must run out (diagnostic).
 cudaError_t launch_wait_selftest(long long limit_cycles, cudaStream_t stream);

@@ -828,11 +828,7 @@ extern "C" int losa_select_noalloc(const float* mass, int B, int H, int n_blocks
   const int64_t R = int64_t(B) * H * n_blocks;
   if (R > kNoallocMaxRows) return LOSA_ERR_ARG;
   if (!(tau > 0.0 && tau <= 1.0) || col_capacity < 0) return LOSA_ERR_ARG;
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return LOSA_ERR_CUDA;
-  if (major != 10) return LOSA_ERR_UNSUPPORTED;
+  if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
   unsigned char* scratch = noalloc_scratch();
   int* status = device_status_word();
   if (!scratch || !status) return LOSA_ERR_CUDA;

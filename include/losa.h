@@ -46,8 +46,9 @@
  *     word (set by a kernel that ran out of a bounded wait, or by a bad mass
  *     value), one stream-ordered memory pool (patterns and scratch), the
  *     fixed scratch array of losa_select_noalloc, and its CUDA function
- *     handles. Calls on different streams are independent, except that
- *     overlapping losa_select_noalloc calls share that scratch array.
+ *     handles; and, per process, the wait limit of losa_set_wait_limit.
+ *     Calls on different streams are independent, except that overlapping
+ *     losa_select_noalloc calls share that scratch array.
  */
 #ifndef LOSA_H_
 #define LOSA_H_
@@ -236,10 +237,15 @@ int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, 
  * that array, so calls that overlap on the GPU (on different streams, or
  * from different threads) race and must be serialised by the caller. The
  * first call on a device looks up the array's device address; make that
- * first call before any stream capture. The call does not synchronise: a
- * bad mass value is reported by the next losa_check_status.
+ * first call before any stream capture. The call does not synchronise, so a
+ * bad mass value (NaN, Inf, negative or >= 2) cannot be returned: it raises
+ * the device status word, which the caller reads and clears with
+ * losa_check_status (LOSA_ERR_MASS) after the call. Until it is cleared, the
+ * next losa_select on that device reports LOSA_ERR_MASS too, whatever its
+ * own input, so check the status before the next losa_select.
  * Returns LOSA_OK, LOSA_ERR_ARG (null pointer, sizes, tau outside (0, 1],
- * col_capacity < 0), LOSA_ERR_UNSUPPORTED or LOSA_ERR_CUDA.
+ * col_capacity < 0), LOSA_ERR_UNSUPPORTED (not an sm_100 device) or
+ * LOSA_ERR_CUDA.
  */
 int losa_select_noalloc(const float* mass, int B, int H, int n_blocks, double tau,
                         int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
@@ -255,9 +261,26 @@ void losa_free(losa_pattern* p);
  * losa_check_status - synchronises `stream`, then reads and clears the
  * device status word of the current device. Returns LOSA_ERR_TIMEOUT when a
  * kernel since the last check gave up a bounded wait (its outputs are then
- * undefined), else LOSA_OK or LOSA_ERR_CUDA.
+ * undefined), LOSA_ERR_MASS when a losa_select_noalloc call since the last
+ * check met a bad mass value (its outputs are then undefined), else LOSA_OK
+ * or LOSA_ERR_CUDA. The word records the first event only.
  */
 int losa_check_status(void* stream);
+
+/*
+ * losa_set_wait_limit - diagnostic of the attention kernels' failure path:
+ * sets, for the whole process, how many SM cycles a wait inside the
+ * attention kernels spins before it gives up (1 <= limit_cycles <= 2^33),
+ * or restores the default (about 2 s at the B200's clock) when limit_cycles
+ * is 0. It applies to the losa_dense_mass and losa_sparse_attn launches made
+ * after the call. A kernel whose wait runs out records LOSA_ERR_TIMEOUT in
+ * the device status word, and every warp of the CTA then leaves its loop,
+ * lets the copies and MMAs it issued finish, frees its tensor memory and
+ * returns, so the CUDA context stays usable. With a limit of a few cycles a
+ * launch times out on purpose (its outputs are then undefined). Not for use
+ * while other threads launch. Returns LOSA_ERR_ARG for a limit out of range.
+ */
+int losa_set_wait_limit(int64_t limit_cycles);
 
 /*
  * losa_selftest_wait - diagnostic of the failure path every kernel uses:

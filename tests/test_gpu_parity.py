@@ -198,12 +198,14 @@ def test_tau_one_keeps_every_positive_block_and_equals_dense(losa):
     assert pat.nnz == int((x > 0).sum())
     o2, lse2 = losa.sparse_attn(q, k, v, L, pat)
     torch.cuda.synchronize()
-    if pat.nnz == pat.rows * pat.n_blocks:
-        # every block kept: the sparse kernel computes the dense result
-        q64, k64, v64 = (t.double().cpu().numpy() for t in (q, k, v))
-        o_ref, lse_ref = O.dense_attention(q64, k64, v64, L, 1 / math.sqrt(wl.head_dim))
-        assert_o_close(o2, o_ref, L, what="tau=1 sparse O")
-        assert_lse_close(lse2, lse_ref, L)
+    # These inputs give every block a positive mass (the smallest is ~1e-6,
+    # far above 2^-49), so tau = 1 keeps every block and the sparse kernel
+    # must compute the dense result.
+    assert pat.nnz == pat.rows * pat.n_blocks
+    q64, k64, v64 = (t.double().cpu().numpy() for t in (q, k, v))
+    o_ref, lse_ref = O.dense_attention(q64, k64, v64, L, 1 / math.sqrt(wl.head_dim))
+    assert_o_close(o2, o_ref, L, what="tau=1 sparse O")
+    assert_lse_close(lse2, lse_ref, L)
 
 
 def test_one_hot_mass_rows_keep_one_block(losa):
@@ -307,3 +309,41 @@ def test_bounded_wait_reports_timeout_and_context_survives(losa):
     torch.cuda.synchronize()
     losa.check_status()
     assert torch.allclose(mass.sum(-1), torch.ones_like(mass.sum(-1)), atol=1e-4)
+
+
+def test_attention_kernels_abort_on_a_short_wait_limit(losa):
+    """The attention kernels' own failure path: with a wait limit of one SM
+    cycle, the first wait of the construction and of the sparse kernel that
+    is not satisfied at once gives up; the call reports LOSA_ERR_TIMEOUT
+    through the status word, every warp leaves, the copies and MMAs in
+    flight land, tensor memory is freed, and the next normal calls give
+    bit for bit what they gave before."""
+    lib = losa.lib()
+    wl = W.custom("abort", 4, 128, (2, 16, 64), 64, amplitude=1.2, seed=17)
+    q, k, v = (t.cuda() for t in W.generate(wl, dtype=torch.bfloat16))
+    L, b = wl.seq_len, wl.block
+    losa.check_status()
+    o_ref, lse_ref, mass_ref = losa.dense_mass(q, k, v, L, b)
+    pat = losa.select(mass_ref, b, 0.95)
+    o2_ref, lse2_ref = losa.sparse_attn(q, k, v, L, pat)
+    torch.cuda.synchronize()
+    losa.check_status()
+    assert lib.losa_set_wait_limit(-1) == -1
+    try:
+        losa.set_wait_limit(1)
+        losa.dense_mass(q, k, v, L, b)
+        with pytest.raises(losa.LosaError) as e:
+            losa.check_status()
+        assert e.value.status == -4          # LOSA_ERR_TIMEOUT
+        losa.sparse_attn(q, k, v, L, pat)
+        with pytest.raises(losa.LosaError) as e:
+            losa.check_status()
+        assert e.value.status == -4
+    finally:
+        losa.set_wait_limit(0)               # back to the default
+    o, lse, mass = losa.dense_mass(q, k, v, L, b)
+    o2, lse2 = losa.sparse_attn(q, k, v, L, pat)
+    torch.cuda.synchronize()
+    losa.check_status()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref) and torch.equal(mass, mass_ref)
+    assert torch.equal(o2, o2_ref) and torch.equal(lse2, lse2_ref)

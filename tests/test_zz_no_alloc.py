@@ -66,6 +66,99 @@ def test_noalloc_select_matches_select_on_two_calls(losa):
         pat.close()
 
 
+def _random_mass(H, n, seed):
+    """Mass rows of n key blocks with ties (every 5th block shares one
+    value), exact zeros and a heavy tail, each row summing to ~1 in fp32."""
+    g = torch.Generator().manual_seed(seed)
+    m = torch.rand(1, H, n, n, generator=g, dtype=torch.float64) ** 8
+    m[..., ::5] = m[..., 1:2]
+    m[..., 3::11] = 0.0
+    m = m / m.sum(-1, keepdim=True)
+    return m.to(torch.float32).cuda().contiguous()
+
+
+def _same_as_select(losa, mass, tau):
+    pat = losa.select(mass, 64, tau)
+    ref = pat.export("cpu")
+    st, row_ptr, col_idx, ret, tot = _noalloc(losa, mass, tau)
+    assert st == 0, losa.lib().losa_strerror(st)
+    torch.cuda.synchronize()
+    losa.check_status()
+    nnz = int(row_ptr[-1].item())
+    assert nnz == pat.nnz
+    assert torch.equal(row_ptr.cpu(), ref["row_ptr"])
+    assert torch.equal(col_idx[:nnz].cpu(), ref["col_idx"])
+    assert torch.equal(ret.cpu(), ref["retained_fx"])
+    assert torch.equal(tot.cpu(), ref["total_fx"])
+    pat.close()
+    return nnz
+
+
+def test_noalloc_long_rows_take_the_bucketed_cut(losa):
+    """Rows of more than 512 key blocks go through the bucketed cut kernel;
+    two calls in a row, each bit-exact against losa_select."""
+    _same_as_select(losa, _random_mass(2, 1500, seed=3), 0.99)
+    _same_as_select(losa, _random_mass(1, 2047, seed=4), 0.95)
+
+
+def test_noalloc_truncates_at_col_capacity(losa):
+    """With col_capacity below the number of kept blocks, the row offsets
+    are still complete, the first col_capacity entries are the full list's,
+    and nothing past col_capacity is written."""
+    mass = _random_mass(3, 600, seed=5)
+    full = _same_as_select(losa, mass, 0.99)
+    cap = full // 2
+    B, H, n, _ = mass.shape
+    R = B * H * n
+    row_ptr = torch.full((R + 1,), -7, dtype=torch.int32, device="cuda")
+    col_idx = torch.full((cap + 4096,), -7, dtype=torch.int32, device="cuda")
+    ret = torch.empty(R, dtype=torch.int64, device="cuda")
+    tot = torch.empty(R, dtype=torch.int64, device="cuda")
+    st = losa.lib().losa_select_noalloc(
+        mass.data_ptr(), B, H, n, ctypes.c_double(0.99), row_ptr.data_ptr(),
+        col_idx.data_ptr(), ctypes.c_int64(cap), ret.data_ptr(), tot.data_ptr(),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    losa.check_status()
+    pat = losa.select(mass, 64, 0.99)
+    ref = pat.export("cpu")
+    assert int(row_ptr[-1].item()) == full
+    assert torch.equal(row_ptr.cpu(), ref["row_ptr"])
+    assert torch.equal(col_idx[:cap].cpu(), ref["col_idx"][:cap])
+    assert torch.all(col_idx[cap:] == -7).item()
+    pat.close()
+
+
+def test_noalloc_call_allocates_no_device_memory(losa):
+    """After a first call (which loads the kernels and looks up the scratch
+    array), a call leaves the device's free memory exactly as it was."""
+    mass = _random_mass(2, 300, seed=6)
+    B, H, n, _ = mass.shape
+    R = B * H * n
+    bufs = [torch.empty(R + 1, dtype=torch.int32, device="cuda"),
+            torch.empty(R * n, dtype=torch.int32, device="cuda"),
+            torch.empty(R, dtype=torch.int64, device="cuda"),
+            torch.empty(R, dtype=torch.int64, device="cuda")]
+
+    def call():
+        st = losa.lib().losa_select_noalloc(
+            mass.data_ptr(), B, H, n, ctypes.c_double(0.99), bufs[0].data_ptr(),
+            bufs[1].data_ptr(), ctypes.c_int64(R * n), bufs[2].data_ptr(), bufs[3].data_ptr(),
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == 0
+        torch.cuda.synchronize()
+
+    call()
+    free0, _ = torch.cuda.mem_get_info()
+    reserved0 = torch.cuda.memory_reserved()
+    call()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_reserved() == reserved0
+    losa.check_status()
+
+
 def test_noalloc_rejects_rows_beyond_its_scratch(losa):
     mass = torch.zeros(1, 1, 8, 8, device="cuda")
     out = torch.zeros(16, dtype=torch.int64, device="cuda")
