@@ -4,9 +4,11 @@
 One step = one pass of the whole hot path over one layer of synthetic input:
 the construction step (dense attention + exact block masses, one kernel),
 the selection (frozen CSR pattern), then the workload's sparse steps on
-freshly drifted Q/K/V (10 for the Wan2.1-1.3B-shaped layer). The timed
-region holds K such steps with every input already resident in HBM; the
-inputs of one step (3.3 GB at the default workload) exceed the 126 MB L2.
+freshly drifted Q/K/V (40 for the default HunyuanVideo-shaped layer: 24
+heads, 118,912 tokens, d 128, block 128; 10 for the Wan2.1-1.3B-shaped one).
+The timed region holds K such steps with every input already resident in
+HBM; the inputs of one call (2.2 GB at the default workload) exceed the
+126 MB L2.
 
 value = algorithmic TFLOP/s of the step:
   construction pass 6*B*H*L_pad^2*d  (Q K^T twice and P V once),
@@ -39,7 +41,7 @@ import workloads as W  # noqa: E402
 
 METRIC = ("block-sparse attn ms & TFLOP/s (retained blocks), % BF16 TC peak; "
           "mass+select ms")
-DEFAULT_WORKLOAD = "wan2.1-1.3b"
+DEFAULT_WORKLOAD = "hunyuanvideo"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Kernels the library launches per call: dense_mass 1 (bf16 inputs), select 8, sparse 1.
 LAUNCHES_DENSE, LAUNCHES_SELECT, LAUNCHES_SPARSE = 1, 8, 1
@@ -61,6 +63,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ncu-case", action="store_true",
                     help="only run dense_mass x2, select, sparse_attn x2 (profiling)")
+    ap.add_argument("--ncu-select", action="store_true",
+                    help="build the mass map, free everything else, run select x2 (profiling)")
     ap.add_argument("--tau-sweep", action="store_true",
                     help="per tau: kept fraction, sparse vs dense time, output error vs dense")
     ap.add_argument("--stability", action="store_true",
@@ -168,21 +172,36 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle sample
 
-def oracle_sample(wl, tau, n_sparse, budget_s, seed=4321):
+_ORACLE_INPUTS = {}
+
+
+def _oracle_inputs(wl, n_sets):
+    """Head 0 of the workload (construction Q/K/V and up to n_sets distinct
+    drifted sets) as fp64 host arrays, drawn once per process."""
+    key = (wl.name, n_sets)
+    if key not in _ORACLE_INPUTS:
+        wl1 = dataclasses.replace(wl, heads=1, batch=1)
+        q, k, v = W.generate(wl1, dtype=torch.float32)
+        sets, prev = [], (q, k, v)
+        for s in range(n_sets):
+            prev = W.drift(wl1, prev, step=s + 1, dtype=torch.float32)
+            sets.append(tuple(t[0, 0].double().numpy() for t in prev))
+        _ORACLE_INPUTS[key] = (tuple(t[0, 0].double().numpy() for t in (q, k, v)), sets)
+    return _ORACLE_INPUTS[key]
+
+
+def oracle_sample(wl, tau, n_sparse, budget_s, seed=4321, max_sets=4):
     """Times the oracle on a bounded sample of the workload: whole query
-    blocks of head 0 (dense rows, mass row, selection, and the sparse steps
-    of that block), until `budget_s` of CPU time. Returns (flops, seconds,
-    blocks, threads)."""
+    blocks of head 0 (dense rows, mass row, selection, and n_sparse sparse
+    steps of that block, cycling through up to max_sets distinct drifted
+    inputs), until `budget_s` of CPU time. Returns (flops, seconds, blocks,
+    threads)."""
     import numpy as np
     import oracle as O
-    wl1 = dataclasses.replace(wl, heads=1, batch=1)
-    q, k, v = W.generate(wl1, dtype=torch.float32)
-    drifts = [W.drift(wl1, (q, k, v), step=s + 1, dtype=torch.float32) for s in range(n_sparse)]
+    (qh, kh, vh), dh = _oracle_inputs(wl, max(1, min(n_sparse, max_sets)))
     L, Lp, b, d = wl.seq_len, wl.seq_pad, wl.block, wl.head_dim
     scale = 1.0 / math.sqrt(d)
-    qh, kh, vh = (t[0, 0].double().numpy() for t in (q, k, v))
     q4, k4 = qh[None, None], kh[None, None]
-    dh = [tuple(t[0, 0].double().numpy() for t in s) for s in drifts]
     g = np.random.default_rng(seed)
     order = g.permutation(wl.n_blocks)
     flops, blocks = 0.0, 0
@@ -193,7 +212,8 @@ def oracle_sample(wl, tau, n_sparse, budget_s, seed=4321):
         m = O.block_mass_row(q4, k4, L, b, scale, 0, 0, int(I))
         kept, _, _ = O.select_row(O.to_fixed(m.astype(np.float32)).tolist(), tau)
         keys = O.retained_keys(kept, b, L)
-        for (q2, k2, v2) in dh:
+        for s in range(n_sparse):
+            q2, k2, v2 = dh[s % len(dh)]
             O.attention_rows(q2[rows], k2[keys], v2[keys], scale)
         flops += 6.0 * b * Lp * d + n_sparse * 4.0 * b * b * d * len(kept)
         blocks += 1
@@ -207,6 +227,24 @@ def oracle_sample(wl, tau, n_sparse, budget_s, seed=4321):
     except Exception:
         pass
     return flops, secs, blocks, threads
+
+
+def distinct_sets(wl, n_sparse):
+    """How many distinct drifted input sets stay resident (at most ~16 GB);
+    longer runs cycle through them."""
+    set_bytes = 3 * wl.batch * wl.heads * wl.seq_pad * wl.head_dim * 2
+    return max(1, min(n_sparse, int(16e9 // set_bytes)))
+
+
+def bench_config(wl, tau, n_sparse, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    B, H, Lp, d = wl.batch, wl.heads, wl.seq_pad, wl.head_dim
+    return {"workload": wl.name, "batch": B, "heads": H, "head_dim": d,
+            "seq_len": wl.seq_len, "seq_pad": Lp, "block": wl.block, "tau": tau,
+            "sparse_steps": n_sparse, "distinct_step_inputs": distinct_sets(wl, n_sparse),
+            "l2": "inputs larger than L2 (3 x "
+                  f"{B * H * Lp * d * 2 / 1e6:.0f} MB per call)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 # ------------------------------------------------------------------ distributed
@@ -251,12 +289,16 @@ def reference_arm(args, world, rank):
         return 0
     wl = W.WORKLOADS[args.workload]
     n_sparse = args.sparse_steps if args.sparse_steps is not None else max(1, wl.sparse_steps)
+    # A bounded sample per step: whole query blocks with at most 8 of the
+    # workload's sparse steps each, so that the run ends within minutes.
+    n_sp_sample = min(n_sparse, 8)
     per_step = min(args.cpu_seconds, max(1.0, min(8.0, 120.0 / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
-        oracle_sample(wl, args.tau, n_sparse, per_step / 4)
+        oracle_sample(wl, args.tau, n_sp_sample, per_step / 4)
     tot_f, tot_s, tot_b, threads = 0.0, 0.0, 0, os.cpu_count()
     for s in range(args.steps):
-        f, secs, blocks, threads = oracle_sample(wl, args.tau, n_sparse, per_step, seed=100 + s)
+        f, secs, blocks, threads = oracle_sample(wl, args.tau, n_sp_sample, per_step,
+                                                 seed=100 + s)
         tot_f += f
         tot_s += secs
         tot_b += blocks
@@ -266,13 +308,11 @@ def reference_arm(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": wl.name, "heads": wl.heads, "head_dim": wl.head_dim,
-                   "seq_len": wl.seq_len, "seq_pad": wl.seq_pad, "block": wl.block,
-                   "tau": args.tau, "sparse_steps": n_sparse},
+        "config": bench_config(wl, args.tau, n_sparse, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{tot_b} whole query blocks of head 0 (dense rows, mass "
-                                   f"row, selection, {n_sparse} sparse steps), {per_step:.0f} s "
-                                   f"per step"},
+                                   f"row, selection, {n_sp_sample} sparse steps each), "
+                                   f"{per_step:.1f} s per step"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -394,6 +434,26 @@ def stability(losa, wl, args, dev, tau=0.99):
     return out
 
 
+def ncu_select_case(losa, wl, tau, dev):
+    """Profiling case for the selection kernels: the workload's real mass map
+    from one construction launch, then everything but the map is freed, so
+    the two selection calls run with only the map and the patterns on the
+    device."""
+    L, b = wl.seq_len, wl.block
+    q, k, v = W.generate(wl, device=dev)
+    _, _, mass = losa.dense_mass(q, k, v, L, b, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    del q, k, v
+    torch.cuda.empty_cache()
+    for _ in range(2):
+        losa.select(mass, b, tau).close()
+    torch.cuda.synchronize()
+    losa.check_status()
+    print(f"ncu select case done: {wl.name}, mass map {mass.numel() * 4 / 1e6:.0f} MB",
+          flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ LoSA arm
 
 def main():
@@ -415,6 +475,8 @@ def main():
         if args.stability:
             stability(losa, wl, args, dev)
         return 0
+    if args.ncu_select:
+        return ncu_select_case(losa, wl, args.tau, torch.device("cuda", local))
     n_sparse = args.sparse_steps if args.sparse_steps is not None else max(1, wl.sparse_steps)
     if args.ncu_case:
         n_sparse = 1  # keeps the device footprint of a profiled run small
@@ -426,8 +488,7 @@ def main():
     # all resident. At most ~16 GB of distinct drifted sets are kept; longer
     # runs (HunyuanVideo-shaped: 40 steps) cycle through them.
     qkv0 = W.generate(wl, device=dev)
-    set_bytes = 3 * wl.batch * wl.heads * Lp * d * 2
-    n_sets = max(1, min(n_sparse, int(16e9 // set_bytes)))
+    n_sets = distinct_sets(wl, n_sparse)
     distinct, prev = [], qkv0
     for s in range(n_sets):
         prev = W.drift(wl, prev, step=s + 1, device=dev)
@@ -516,12 +577,7 @@ def main():
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "batch": B, "heads": H, "head_dim": d,
-                   "seq_len": L, "seq_pad": Lp, "block": b, "tau": tau,
-                   "sparse_steps": n_sparse, "distinct_step_inputs": n_sets,
-                   "l2": "inputs larger than L2 (3 x "
-                   f"{B * H * Lp * d * 2 / 1e6:.0f} MB per call)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": bench_config(wl, tau, n_sparse, world),
         "sparse_attn": {"ms": sparse_ms, "tflops": sparse_tf, "frac_of_peak": sparse_tf / peak,
                         "retained_blocks": nnz, "kept_fraction": density,
                         "tile_entries": tile_entries,
@@ -541,7 +597,7 @@ def main():
     }
 
     if not args.no_e2e:
-        line["e2e"] = e2e_measure(losa, wl, qkv0, sets, args, world)
+        line["e2e"] = e2e_measure(losa, wl, qkv0, distinct, n_sparse, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, secs, blocks, threads = oracle_sample(wl, tau, n_sparse, args.cpu_seconds)
         line["cpu_baseline"] = {
@@ -556,30 +612,36 @@ def main():
     return 0
 
 
-def e2e_measure(losa, wl, qkv0, sets, args, world):
+def e2e_measure(losa, wl, qkv0, distinct, n_sparse, args, world, max_host_sets=4):
     """The same step through the public API from pinned HOST buffers: every
     call's inputs are copied host->device and every call's output
     device->host inside the timed region. Host->device and device->host
     copies run on two streams of their own (PCIe carries both directions at
     once), double-buffered, so call i+1's inputs arrive while call i
-    computes (what a caller streaming activations would do)."""
+    computes (what a caller streaming activations would do). The host holds
+    the construction inputs and up to max_host_sets distinct drifted sets,
+    which the sparse calls cycle through; each call still copies its full
+    inputs, and outputs land in two pinned host buffers in turn."""
     L, Lp, b, d, tau = wl.seq_len, wl.seq_pad, wl.block, wl.head_dim, args.tau
     dev = qkv0[0].device
     comp = torch.cuda.current_stream()
     up = torch.cuda.Stream(device=dev)     # host -> device
     down = torch.cuda.Stream(device=dev)   # device -> host
-    host_sets = [tuple(t.cpu().pin_memory() for t in s) for s in [qkv0] + sets]
-    n_calls = len(host_sets)
+    host_distinct = [tuple(t.cpu().pin_memory() for t in s)
+                     for s in [qkv0] + list(distinct[:max_host_sets])]
+    n_calls = 1 + n_sparse
+    host_in = lambda i: host_distinct[0] if i == 0 else \
+        host_distinct[1 + (i - 1) % (len(host_distinct) - 1)]
     out_host = [torch.empty(wl.batch, wl.heads, Lp, d, dtype=torch.bfloat16).pin_memory()
-                for _ in host_sets]
-    dev_in = [tuple(torch.empty_like(t, device=dev) for t in host_sets[0]) for _ in range(2)]
+                for _ in range(2)]
+    dev_in = [tuple(torch.empty_like(t, device=dev) for t in host_distinct[0]) for _ in range(2)]
     dev_out = [torch.empty(wl.batch, wl.heads, Lp, d, dtype=torch.bfloat16, device=dev)
                for _ in range(2)]
     lse = torch.empty(wl.batch, wl.heads, Lp, dtype=torch.float32, device=dev)
     mass = torch.empty(wl.batch, wl.heads, wl.n_blocks, wl.n_blocks, dtype=torch.float32,
                        device=dev)
-    h2d = sum(t.numel() * t.element_size() for s in host_sets for t in s)
-    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    h2d = sum(t.numel() * t.element_size() for i in range(n_calls) for t in host_in(i))
+    d2h = n_calls * out_host[0].numel() * out_host[0].element_size()
     ev = lambda: torch.cuda.Event()
 
     def step():
@@ -589,15 +651,15 @@ def e2e_measure(losa, wl, qkv0, sets, args, world):
             with torch.cuda.stream(up):
                 if i >= 2:
                     up.wait_event(done[i - 2])
-                for dst, src in zip(dev_in[i % 2], host_sets[i]):
+                for dst, src in zip(dev_in[i % 2], host_in(i)):
                     dst.copy_(src, non_blocking=True)
                 in_ready[i] = ev()
                 in_ready[i].record(up)
 
-        def unload(i):  # output of call i back to the host
+        def unload(i):  # output of call i back to host buffer i % 2 (in order on `down`)
             with torch.cuda.stream(down):
                 down.wait_event(done[i])
-                out_host[i].copy_(dev_out[i % 2], non_blocking=True)
+                out_host[i % 2].copy_(dev_out[i % 2], non_blocking=True)
                 out_free[i] = ev()
                 out_free[i].record(down)
 

@@ -39,6 +39,12 @@ def test_reference_arm_two_ranks():
     assert rec["n_gpus"] == 2 and rec["warmup"] == 1 and rec["config"]["workload"] == "tiny"
     assert rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
+    # the same config object as the GPU arm's line
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    wl = W.WORKLOADS["tiny"]
+    assert rec["config"] == bench.bench_config(wl, 0.99, max(1, wl.sparse_steps), 2)
 
 
 def _worker(rank, port, out):
