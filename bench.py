@@ -61,12 +61,17 @@ def parse_args():
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (small profiling cases)")
     ap.add_argument("--ncu-case", action="store_true",
                     help="only run dense_mass x2, select, sparse_attn x2 (profiling)")
     ap.add_argument("--ncu-select", action="store_true",
                     help="build the mass map, free everything else, run select x2 (profiling)")
     ap.add_argument("--tau-sweep", action="store_true",
                     help="per tau: kept fraction, sparse vs dense time, output error vs dense")
+    ap.add_argument("--sched-analysis", action="store_true",
+                    help="what a persistent tile scheduler could gain over the hardware's "
+                         "in-order CTA dispatch (measured fixed cost + list scheduling)")
     ap.add_argument("--stability", action="store_true",
                     help="frozen pattern vs fresh selections over the drifted steps")
     return ap.parse_args()
@@ -434,6 +439,67 @@ def stability(losa, wl, args, dev, tau=0.99):
     return out
 
 
+def _list_schedule(costs, workers):
+    """Makespan of greedy in-order list scheduling: each job, in order, goes
+    to the worker that becomes free first."""
+    import heapq
+    free = [0.0] * workers
+    heapq.heapify(free)
+    for c in costs:
+        heapq.heappush(free, heapq.heappop(free) + c)
+    return max(free)
+
+
+def sched_analysis(losa, wl, args, dev, tau=0.99):
+    """Upper bound of what a persistent tile scheduler could recover in the
+    sparse kernel, from two measurements and one simulation:
+      * fixed cost: the same kernel on a pattern with one key block per row
+        (the diagonal), i.e. every CTA's setup, Q load, pipeline fill,
+        epilogue and teardown with almost no iterations, against the real
+        pattern's time;
+      * dispatch and pairing: with the real per-tile iteration counts, the
+        hardware's in-order dispatch of two-tile CTAs (a CTA lasts as long as
+        its longer tile) against a persistent kernel whose 2 x #SM tile slots
+        each take the next tile as soon as they are free, both relative to a
+        perfect split of the iterations over the slots.
+    One JSON line."""
+    L, b, d = wl.seq_len, wl.block, wl.head_dim
+    B, H, n = wl.batch, wl.heads, wl.n_blocks
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    qkv = W.generate(wl, device=dev)
+    _, _, mass = losa.dense_mass(*qkv, L, b, out_dtype=torch.bfloat16)
+    pat = losa.select(mass, b, tau)
+    q1 = W.drift(wl, qkv, step=1, device=dev)
+    del qkv
+    o = torch.empty(B, H, wl.seq_pad, d, device=dev, dtype=torch.bfloat16)
+    t_full = _event_ms(lambda: losa.sparse_attn(*q1, L, pat, out_dtype=torch.bfloat16, o=o,
+                                                want_lse=False), n=5, warm=2)
+    R = B * H * n
+    diag = losa.import_pattern(torch.arange(R + 1, dtype=torch.int32),
+                               torch.arange(n, dtype=torch.int32).repeat(B * H), B, H, n, b,
+                               device=dev)
+    t_diag = _event_ms(lambda: losa.sparse_attn(*q1, L, diag, out_dtype=torch.bfloat16, o=o,
+                                                want_lse=False), n=5, warm=2)
+    ex = pat.export("cpu")
+    counts = (ex["tile_ptr"][1:] - ex["tile_ptr"][:-1]).double()
+    epi = max(1, 128 // b)
+    n_it = torch.ceil(counts / epi)[ex["tile_order"].long()].tolist()  # in launch order
+    pairs = [max(n_it[i], n_it[i + 1] if i + 1 < len(n_it) else 0.0)
+             for i in range(0, len(n_it), 2)]
+    ideal = sum(n_it) / (2 * sms)
+    hw = _list_schedule(pairs, sms)
+    persistent = _list_schedule(n_it, 2 * sms)
+    rec = {"analysis": "sched", "workload": wl.name, "sms": sms, "tiles": len(n_it),
+           "ctas": len(pairs), "sparse_ms": t_full, "diag_pattern_ms": t_diag,
+           "fixed_cost_share": t_diag / t_full,
+           "hw_dispatch_loss": hw / ideal - 1.0, "persistent_loss": persistent / ideal - 1.0,
+           "persistent_gain_bound": (t_diag / t_full) + (hw - persistent) / hw}
+    print(json.dumps(rec), flush=True)
+    pat.close()
+    diag.close()
+    return rec
+
+
 def ncu_select_case(losa, wl, tau, dev):
     """Profiling case for the selection kernels: the workload's real mass map
     from one construction launch, then everything but the map is freed, so
@@ -468,12 +534,16 @@ def main():
     import block_sparse_attention_losa_b200 as losa
 
     wl = W.WORKLOADS[args.workload]
-    if args.tau_sweep or args.stability:
+    if args.heads is not None:
+        wl = dataclasses.replace(wl, heads=args.heads)
+    if args.tau_sweep or args.stability or args.sched_analysis:
         dev = torch.device("cuda", local)
         if args.tau_sweep:
             tau_sweep(losa, wl, args, dev)
         if args.stability:
             stability(losa, wl, args, dev)
+        if args.sched_analysis:
+            sched_analysis(losa, wl, args, dev)
         return 0
     if args.ncu_select:
         return ncu_select_case(losa, wl, args.tau, torch.device("cuda", local))

@@ -128,19 +128,22 @@ int64_t validate_csr(const int32_t* row_ptr, const int32_t* col_idx, int BH, int
   return entries;
 }
 
-// bf16 views of fp32 inputs, converted on the stream into temporaries.
-struct Bf16Inputs {
+// The operands the kernels read: bf16 inputs as given, or fp32 inputs
+// rounded to tf32 (nearest even) on the stream into pool temporaries, for the
+// kind::tf32 kernels.
+struct KernelInputs {
   const void* q;
   const void* k;
   const void* v;
+  bool tf32 = false;
   void* tmp = nullptr;
   cudaStream_t s;
-  ~Bf16Inputs() {
+  ~KernelInputs() {
     if (tmp) cudaFreeAsync(tmp, s);
   }
 };
 
-int prepare_inputs(Bf16Inputs& in, const void* q, const void* k, const void* v, int in_dtype,
+int prepare_inputs(KernelInputs& in, const void* q, const void* k, const void* v, int in_dtype,
                    int64_t n_elem) {
   if (in_dtype == LOSA_BF16) {
     in.q = q;
@@ -148,17 +151,18 @@ int prepare_inputs(Bf16Inputs& in, const void* q, const void* k, const void* v, 
     in.v = v;
     return LOSA_OK;
   }
-  const size_t bytes = size_t(n_elem) * 2;
+  const size_t bytes = size_t(n_elem) * 4;
   in.tmp = pool_alloc(3 * bytes, in.s);
   if (!in.tmp) return LOSA_ERR_NOMEM;
-  char* base = static_cast<char*>(in.tmp);
-  if (launch_f32_to_bf16(static_cast<const float*>(q), base, n_elem, in.s) != cudaSuccess ||
-      launch_f32_to_bf16(static_cast<const float*>(k), base + bytes, n_elem, in.s) != cudaSuccess ||
-      launch_f32_to_bf16(static_cast<const float*>(v), base + 2 * bytes, n_elem, in.s) != cudaSuccess)
+  float* base = static_cast<float*>(in.tmp);
+  if (launch_f32_to_tf32(static_cast<const float*>(q), base, n_elem, in.s) != cudaSuccess ||
+      launch_f32_to_tf32(static_cast<const float*>(k), base + n_elem, n_elem, in.s) != cudaSuccess ||
+      launch_f32_to_tf32(static_cast<const float*>(v), base + 2 * n_elem, n_elem, in.s) != cudaSuccess)
     return LOSA_ERR_CUDA;
   in.q = base;
-  in.k = base + bytes;
-  in.v = base + 2 * bytes;
+  in.k = base + n_elem;
+  in.v = base + 2 * n_elem;
+  in.tf32 = true;
   return LOSA_OK;
 }
 
@@ -179,12 +183,12 @@ int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype, i
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_ARG;
   if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  Bf16Inputs in;
+  KernelInputs in;
   in.s = s;
   const int64_t n_elem = int64_t(B) * H * L_pad * d;
   int st = prepare_inputs(in, q, k, v, in_dtype, n_elem);
   if (st != LOSA_OK) return st;
-  if (launch_dense(in.q, in.k, in.v, B * H, L, L_pad, d, block, scale, o,
+  if (launch_dense(in.q, in.k, in.v, in.tf32, B * H, L, L_pad, d, block, scale, o,
                    out_dtype == LOSA_BF16, lse, mass, s) != cudaSuccess)
     return LOSA_ERR_CUDA;
   return LOSA_OK;
@@ -275,13 +279,13 @@ int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_ARG;
   if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  Bf16Inputs in;
+  KernelInputs in;
   in.s = s;
   const int64_t n_elem = int64_t(p->B) * p->H * L_pad * d;
   int st = prepare_inputs(in, q, k, v, in_dtype, n_elem);
   if (st != LOSA_OK) return st;
-  if (launch_sparse(in.q, in.k, in.v, d, L, scale, p, o, out_dtype == LOSA_BF16, lse, s) !=
-      cudaSuccess)
+  if (launch_sparse(in.q, in.k, in.v, in.tf32, d, L, scale, p, o, out_dtype == LOSA_BF16, lse,
+                    s) != cudaSuccess)
     return LOSA_ERR_CUDA;
   return LOSA_OK;
 }

@@ -53,12 +53,14 @@ struct AttnParams {
   long long wait_limit;   // SM cycles a wait spins before it gives up
 };
 
-template <int D, int BN, int NSK, int NSV>
+// ESZ: bytes per operand element (2 = bf16, 4 = fp32 read as tf32). Every
+// tile is stored as 128-byte-wide slabs (128 / ESZ columns each).
+template <int D, int BN, int NSK, int NSV, int ESZ = 2>
 struct AttnLayout {
   static constexpr int BM = 128;
   static constexpr int NT = 2;                           // query tiles per CTA
-  static constexpr int Q_BYTES = BM * D * 2;             // one tile: D/64 slabs of 16 KB
-  static constexpr int KV_BYTES = BN * D * 2;            // D/64 slabs of BN*128 B
+  static constexpr int Q_BYTES = BM * D * ESZ;           // one tile: D*ESZ/128 slabs of 16 KB
+  static constexpr int KV_BYTES = BN * D * ESZ;          // D*ESZ/128 slabs of BN*128 B
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
@@ -97,22 +99,32 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kAttnThreads * kAtt
               "register split must use exactly the launch allocation");
 
 // BLK: the LoSA block size b (compile time, so that every per-block array
-// stays in registers). Dense: key tiles of BN = 128 rows, one TMA box each;
-// the mass pass sums over b x b blocks. Sparse: each 128-key iteration packs
-// EPI = BN / b consecutive entries of the tile's list into one K/V stage
-// (one b-row box each, stacked), so the tensor core always runs N = 128.
-template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK>
+// stays in registers). Dense: key tiles of BN rows, one TMA box each; the
+// mass pass sums over b x b blocks (a block wider than a key tile is summed
+// over CPE consecutive tiles). Sparse: each BN-key iteration packs EPI =
+// BN / b consecutive entries of the tile's list into one K/V stage (one b-row
+// box each, stacked), so the tensor core runs N = BN; an entry wider than BN
+// takes CPE = b / BN iterations.
+// kTf32: Q, K, V are fp32 (already rounded to tf32) and every MMA is
+// kind::tf32; the weights P stay fp32 in TMEM as the tf32 A operand of P V.
+template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK, bool kTf32>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using Lay = AttnLayout<D, BN, NSK, NSV>;
+  constexpr int ESZ = kTf32 ? 4 : 2;       // bytes per operand element
+  using Lay = AttnLayout<D, BN, NSK, NSV, ESZ>;
   constexpr int BM = Lay::BM;
-  constexpr int N_SLABS = D / 64;
-  constexpr int BOX = kDense ? BN : BLK;  // key rows per TMA box
-  constexpr int EPI = BN / BOX;           // boxes (list entries) per key stage
-  static_assert(BN % BLK == 0 && BLK % 32 == 0, "block size");
-  constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
-  constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+  constexpr int SLAB_COLS = 128 / ESZ;     // operand columns per 128-byte slab
+  constexpr int N_SLABS = D / SLAB_COLS;
+  constexpr int BOX = kDense ? BN : (BLK < BN ? BLK : BN);  // key rows per TMA box
+  constexpr int EPI = BN / BOX;            // boxes (list entries) per key stage
+  constexpr int CPE = BLK > BN ? BLK / BN : 1;  // key stages per list entry / key block
+  constexpr int K_STEP = 32 / ESZ;         // K of one MMA instruction (32 bytes of a row)
+  static_assert((BN % BLK == 0 || BLK % BN == 0) && BLK % 32 == 0, "block size");
+  constexpr uint32_t IDESC_S = kTf32 ? idesc_tf32_f32(BM, BN, false, false)
+                                     : idesc_bf16_f32(BM, BN, false, false);
+  constexpr uint32_t IDESC_PV = kTf32 ? idesc_tf32_f32(BM, D, false, true)
+                                      : idesc_bf16_f32(BM, D, false, true);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -156,7 +168,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         qt[t] = tile - bh[t] * p.n_qt;
         e_begin[t] = p.tile_ptr[tile];
         n_ent[t] = p.tile_ptr[tile + 1] - e_begin[t];
-        n_it[t] = (n_ent[t] + EPI - 1) / EPI;
+        n_it[t] = CPE * ((n_ent[t] + EPI - 1) / EPI);
       } else {
         bh[t] = 0;
         qt[t] = 0;
@@ -207,12 +219,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive_expect_tx(&q_full[t], Lay::Q_BYTES);
 #pragma unroll
         for (int s = 0; s < N_SLABS; ++s)
-          tma_load_3d(sQ + t * Lay::Q_BYTES + s * (BM * 128), &tm_q, &q_full[t], s * 64,
-                      qt[t] * BM, bh[t]);
+          tma_load_3d(sQ + t * Lay::Q_BYTES + s * (BM * 128), &tm_q, &q_full[t],
+                      s * SLAB_COLS, qt[t] * BM, bh[t]);
       }
       int kc = 0, vc = 0;
       bool ok = true;
-      // One stage = BN keys = EPI boxes of BLK rows, stacked in each slab.
+      // One stage = BN keys = EPI boxes of BOX rows, stacked in each slab.
       auto load_k = [&](const int (&key_row)[EPI], int head) -> bool {
         const int ks = kc % NSK;
         if (!mbar_wait(&k_empty[ks], ((kc / NSK) & 1) ^ 1, wc)) return false;
@@ -222,7 +234,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int e = 0; e < EPI; ++e)
             tma_load_3d(sK + ks * Lay::KV_BYTES + s * (BN * 128) + e * (BOX * 128), &tm_k,
-                        &k_full[ks], s * 64, key_row[e], head);
+                        &k_full[ks], s * SLAB_COLS, key_row[e], head);
         ++kc;
         return true;
       };
@@ -235,7 +247,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int e = 0; e < EPI; ++e)
             tma_load_3d(sV + vs * Lay::KV_BYTES + s * (BN * 128) + e * (BOX * 128), &tm_v,
-                        &v_full[vs], s * 64, key_row[e], head);
+                        &v_full[vs], s * SLAB_COLS, key_row[e], head);
         ++vc;
         return true;
       };
@@ -254,12 +266,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (ok && j < n_it[t]) {
+              // Box e of iteration j: list entry j * EPI + e, or, for an
+              // entry wider than a stage, chunk j % CPE of entry j / CPE.
               // Slots past the end of the list repeat its last entry (valid,
               // finite data); the softmax masks those columns.
               int rows[EPI];
 #pragma unroll
-              for (int e = 0; e < EPI; ++e)
-                rows[e] = (p.tile_entry[e_begin[t] + min(j * EPI + e, n_ent[t] - 1)] & 0xFFFF) * BLK;
+              for (int e = 0; e < EPI; ++e) {
+                const int idx = CPE > 1 ? j / CPE : j * EPI + e;
+                rows[e] = (p.tile_entry[e_begin[t] + min(idx, n_ent[t] - 1)] & 0xFFFF) * BLK +
+                          (CPE > 1 ? (j % CPE) * BN : 0);
+              }
               ok = load_k(rows, bh[t]) && load_v(rows, bh[t]);
             }
           }
@@ -300,12 +317,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const uint32_t qb = q_base + t * Lay::Q_BYTES;
         const uint32_t d_tmem = tmem + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
+        // 32 bytes of K per instruction: four steps per 128-byte slab.
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / K_STEP; ++kk) {
           const uint64_t a = sdesc_sw128(qb + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
           const uint64_t b = sdesc_sw128(k_base + ks * Lay::KV_BYTES + (kk >> 2) * (BN * 128) +
                                              (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+          if constexpr (kTf32)
+            umma_tf32_ss(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+          else
+            umma_bf16_ss(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[t]);
         return true;
@@ -324,10 +345,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const uint32_t a_tmem = tmem + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
         const uint32_t d_tmem = tmem + (t ? Lay::TMEM_O1 : Lay::TMEM_O0);
+        // K_STEP keys per instruction: 8 TMEM columns of P (two bf16 or one
+        // fp32 per column) and K_STEP 128-byte rows of V. V is the MN-major
+        // operand: 128-byte swizzle (8-row groups 1 KB apart) for bf16, the
+        // 32-byte-atom 128-byte swizzle (4-row groups 512 B apart) for tf32.
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t b = sdesc_sw128(v_base + vs * Lay::KV_BYTES + kk * 2048, BN * 128, 1024);
-          umma_bf16_ts(d_tmem, a_tmem + kk * 8, b, IDESC_PV, (pc[t] > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / K_STEP; ++kk) {
+          const uint32_t vaddr = v_base + vs * Lay::KV_BYTES + kk * (K_STEP * 128);
+          if constexpr (kTf32)
+            umma_tf32_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128_32b(vaddr, BN * 128, 512), IDESC_PV,
+                         (pc[t] > 0 || kk > 0) ? 1u : 0u);
+          else
+            umma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(vaddr, BN * 128, 1024), IDESC_PV,
+                         (pc[t] > 0 || kk > 0) ? 1u : 0u);
         }
         ++pc[t];
         return true;
@@ -454,7 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int e = 0; e < EPI; ++e) {
           ent[e] = ent_next[e];
-          const int idx = (j + 1) * EPI + e;
+          const int idx = CPE > 1 ? (j + 1) / CPE : (j + 1) * EPI + e;
           ent_next[e] = (idx < n) ? __ldg(p.tile_entry + e_begin[t] + idx) : 0;
         }
       }
@@ -484,12 +514,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int qb = r / BLK;
 #pragma unroll
         for (int e = 0; e < EPI; ++e) {
-          const int key0 = (ent[e] & 0xFFFF) * BLK;
+          const int key0 = (ent[e] & 0xFFFF) * BLK + (CPE > 1 ? (j % CPE) * BN : 0);
           on[e] = ((ent[e] >> 16) >> qb) & 1;
-          if (key0 + BLK > p.L) {
+          if (key0 + BOX > p.L) {
 #pragma unroll
-            for (int c = 0; c < BLK; ++c)
-              if (key0 + c >= p.L) s[e * BLK + c] = NEG_INF;
+            for (int c = 0; c < BOX; ++c)
+              if (key0 + c >= p.L) s[e * BOX + c] = NEG_INF;
           }
         }
       }
@@ -535,9 +565,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // row sum in packed adds.
       const f32x2 sl2x2 = f2_make(sl2, sl2);
       f32x2 ts2[2] = {0ull, 0ull};
+      // The weights go over S_t chunk by chunk (S is in registers by now):
+      // bf16, 16 packed pairs per 32 columns, or, in the tf32 kernels, fp32,
+      // one column per key.
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t pk[16];
+        float pf[kTf32 ? 32 : 1];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const float ns = nsub[(c * 32 + g * 8) / BOX];
@@ -554,10 +588,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               e1 = ex2_approx(a1);
             }
             ts2[i & 1] = f2_add(ts2[i & 1], f2_make(e0, e1));
-            pk[g * 4 + i] = pack_bf16x2(e0, e1);
+            if constexpr (kTf32) {
+              pf[g * 8 + 2 * i] = e0;
+              pf[g * 8 + 2 * i + 1] = e1;
+            } else {
+              pk[g * 4 + i] = pack_bf16x2(e0, e1);
+            }
           }
         }
-        tmem_st16(s_col + c * 16, pk);
+        if constexpr (kTf32)
+          tmem_st32(s_col + c * 32, pf);
+        else
+          tmem_st16(s_col + c * 16, pk);
       }
       if (rescale) {
         // O_t *= alpha. S_t(j) completing implies PV_t(j-1) completed, so
@@ -632,7 +674,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if constexpr (kDense) {
       // ---- pass 2: block masses from exp(s - lse)
-      constexpr int NKB = BN / BLK;      // key blocks per key tile
+      constexpr int NKB = BN >= BLK ? BN / BLK : 1;  // key blocks per key tile
       constexpr int NG = BN / 32;        // 32-column groups per key tile
       constexpr int WPB = BLK / 32;      // warps per query block (1, 2 or 4)
       const int q_local = r / BLK;       // query block within the tile
@@ -641,6 +683,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float inv_cnt = (n_valid_I > 0) ? 1.f / float(n_valid_I) : 0.f;
       const float lsub = row_valid ? lse2 : __int_as_float(0x7f800000);
       float* red_t = red + t * 32;
+      float carry = 0.f;  // a key block over CPE key tiles: the earlier tiles' sum
       for (int j = 0; ok && j < n_iter; ++j) {
         if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
         ++sc;
@@ -708,6 +751,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int off = 16; off > 0; off >>= 1)
             kbsum[kb] += __shfl_xor_sync(0xffffffffu, kbsum[kb], off);
         }
+        if constexpr (CPE > 1) {
+          // This tile is chunk j % CPE of one key block: carry the sum until
+          // the block's last chunk.
+          kbsum[0] += carry;
+          if (j % CPE != CPE - 1) {
+            carry = kbsum[0];
+            continue;
+          }
+          carry = 0.f;
+        }
+        const int w_idx = j / CPE;         // key blocks written so far (CPE > 1), else j
         const int J0 = key0 / BLK;
         float* mrow = p.mass + (size_t(bh[t]) * p.n_blocks + I) * p.n_blocks;
         if constexpr (WPB == 1) {
@@ -717,13 +771,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               if (J0 + kb < p.n_blocks) mrow[J0 + kb] = kbsum[kb] * inv_cnt;
           }
         } else {
-          float* rb = red_t + (j & 1) * 16;
+          float* rb = red_t + (w_idx & 1) * 16;
           if (lane == 0) {
 #pragma unroll
             for (int kb = 0; kb < NKB; ++kb) rb[wl * 4 + kb] = kbsum[kb];
           }
-          mbar_arrive(&red_bar[2 * t + (j & 1)]);
-          if (!mbar_wait(&red_bar[2 * t + (j & 1)], (j >> 1) & 1, wc)) { ok = false; break; }
+          mbar_arrive(&red_bar[2 * t + (w_idx & 1)]);
+          if (!mbar_wait(&red_bar[2 * t + (w_idx & 1)], (w_idx >> 1) & 1, wc)) { ok = false; break; }
           if (lane == 0 && (wl % WPB) == 0 && I < p.n_blocks) {
 #pragma unroll
             for (int kb = 0; kb < NKB; ++kb) {

@@ -43,13 +43,15 @@ cudaMemPool_t device_pool();
 void* pool_alloc(size_t bytes, cudaStream_t stream);
 
 // Runs the dense two-pass construction kernel. q/k/v are bf16 device
-// pointers; the arguments were validated by the caller.
-cudaError_t launch_dense(const void* q, const void* k, const void* v, int BH, int L, int L_pad,
-                         int d, int block, float scale, void* o, bool out_bf16, float* lse,
-                         float* mass, cudaStream_t stream);
+// pointers, or fp32 ones already rounded to tf32 when tf32 is set; the
+// arguments were validated by the caller.
+cudaError_t launch_dense(const void* q, const void* k, const void* v, bool tf32, int BH, int L,
+                         int L_pad, int d, int block, float scale, void* o, bool out_bf16,
+                         float* lse, float* mass, cudaStream_t stream);
 
-// Runs the block-sparse kernel over pattern p (validated by the caller).
-cudaError_t launch_sparse(const void* q, const void* k, const void* v, int d, int L,
+// Runs the block-sparse kernel over pattern p (validated by the caller);
+// q/k/v as for launch_dense.
+cudaError_t launch_sparse(const void* q, const void* k, const void* v, bool tf32, int d, int L,
                           float scale, const losa_pattern* p, void* o, bool out_bf16,
                           float* lse, cudaStream_t stream);
 
@@ -65,6 +67,10 @@ cudaError_t launch_exp2_eval(const float* x, float* y, int64_t n, cudaStream_t s
 
 // fp32 -> bf16 (round to nearest even) of n elements.
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
+
+// fp32 -> tf32 (round to nearest even, kept as fp32 with the 13 low mantissa
+// bits zero) of n elements.
+cudaError_t launch_f32_to_tf32(const float* src, float* dst, int64_t n, cudaStream_t stream);
 
 // Builds the frozen pattern from a mass map (validated by the caller).
 // Returns a losa_status.

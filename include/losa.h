@@ -60,8 +60,13 @@ extern "C" {
 #endif
 
 typedef enum {
-  LOSA_BF16 = 0, /* bfloat16 */
-  LOSA_FP32 = 1  /* float32; inputs are rounded to bf16 (nearest even) on entry */
+  LOSA_BF16 = 0, /* bfloat16: the attention runs on kind::f16 tensor cores
+                    (bf16 operands, bf16 weights P, fp32 accumulation) */
+  LOSA_FP32 = 1  /* float32: inputs are rounded to tf32 (nearest even, 10
+                    mantissa bits) on entry into pool temporaries and the
+                    attention runs on kind::tf32 tensor cores (the weights P
+                    stay fp32 and are read as tf32); as an output dtype,
+                    float32 */
 } losa_dtype;
 
 typedef enum {
@@ -103,7 +108,8 @@ typedef struct {
  * attention mass (Phase 1 - Dense Calibration, ubos.tech LoSA post; LoSA
  * abstract).
  *
- *   q, k, v    [B, H, L_pad, d] device, dtype in_dtype.
+ *   q, k, v    [B, H, L_pad, d] device, dtype in_dtype (LOSA_FP32 takes
+ *              the tf32 path: see losa_dtype).
  *   o          [B, H, L_pad, d] device, dtype out_dtype:
  *              O = softmax(scale * Q K^T over keys j < L) V.
  *   lse        [B, H, L_pad] fp32 device: lse_i = log sum_{j<L} exp(scale q_i.k_j).

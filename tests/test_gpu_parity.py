@@ -1,16 +1,22 @@
 """GPU path (through the C ABI) against the CPU oracle, element by element.
 
+Inputs: the oracle is handed the values the library computes on: bf16
+inputs as they are, and fp32 inputs rounded to tf32 (round to nearest even,
+workloads.round_tf32), since the library rounds fp32 inputs to tf32 on entry
+and runs kind::tf32 MMAs on them.
+
 Tolerances, per output:
   * block mass: |delta| <= 1e-5 absolute (fp32 accumulation of exact
-    bf16 x bf16 products; the row sums to 1, so fp32 rounding of the sum
-    and of exp2 stays near 1e-7 per term).
+    bf16 x bf16 or tf32 x tf32 products; the row sums to 1, so fp32 rounding
+    of the sum and of exp2 stays near 1e-7 per term).
   * selection: bit-exact (row_ptr, col_idx, retained_fx, total_fx) against
     the oracle's selection run on the GPU's own fp32 masses; with the
     oracle's fp64 masses, the kept set still holds >= tau - 1e-5 of the mass.
   * O (fp32 output): max |delta| <= 1e-2 and mean |delta| <= 1e-3 against
-    fp64 on the same bf16 inputs. P is rounded to bf16 before the P.V
-    product (relative 2^-9 per weight), which bounds the error near
-    2^-9 * max|v| ~ 0.008 in the worst case and ~1e-4 on average.
+    fp64 on the same rounded inputs. P is rounded to bf16 (tf32 on the fp32
+    path) before the P.V product (relative 2^-9, resp. 2^-11, per weight),
+    which bounds the error near 2^-9 * max|v| ~ 0.008 in the worst case and
+    ~1e-4 on average.
   * O (bf16 output): additionally the output's own rounding, half an ulp:
     |delta| <= 1e-2 + 2^-8 |O|.
   * lse: |delta| <= 1e-4 (fp32 scores of exact products; the sum of exp
@@ -108,6 +114,11 @@ def check_selection(pat, mass_gpu, tau, check_tile_lists=True):
     return ref, ex
 
 
+def computed_on(t, in_fp32):
+    """The values the library computes on for inputs t (fp32 on the host)."""
+    return W.round_tf32(t) if in_fp32 else t.to(torch.bfloat16).to(torch.float32)
+
+
 def run_small(losa, wl, tau=0.99, out_dtype=torch.float32, in_fp32=None):
     q, k, v = W.generate(wl, dtype=torch.float32)
     if in_fp32 is None:
@@ -118,7 +129,7 @@ def run_small(losa, wl, tau=0.99, out_dtype=torch.float32, in_fp32=None):
     o, lse, mass = losa.dense_mass(qd, kd, vd, L, b, out_dtype=out_dtype)
     torch.cuda.synchronize()
     losa.check_status()
-    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
+    q64, k64, v64 = (computed_on(t, in_fp32).double().numpy() for t in (q, k, v))
     o_ref, lse_ref = O.dense_attention(q64, k64, v64, L, scale)
     mass_ref = O.block_mass(q64, k64, L, b, scale)
     assert_o_close(o, o_ref, L, bf16_out=out_dtype == torch.bfloat16, what="dense O")
@@ -140,9 +151,9 @@ def run_small(losa, wl, tau=0.99, out_dtype=torch.float32, in_fp32=None):
     o2, lse2 = losa.sparse_attn(q2d, k2d, v2d, L, pat, out_dtype=out_dtype)
     torch.cuda.synchronize()
     losa.check_status()
-    o2_ref, lse2_ref = O.sparse_attention(q2.double().numpy(), k2.double().numpy(),
-                                          v2.double().numpy(), L, b, scale, ref["row_ptr"],
-                                          ref["col_idx"])
+    o2_ref, lse2_ref = O.sparse_attention(*(computed_on(t, in_fp32).double().numpy()
+                                            for t in (q2, k2, v2)), L, b, scale,
+                                          ref["row_ptr"], ref["col_idx"])
     assert_o_close(o2, o2_ref, L, bf16_out=out_dtype == torch.bfloat16, what="sparse O")
     assert_lse_close(lse2, lse2_ref, L)
     return pat
@@ -183,9 +194,43 @@ def test_bf16_io(losa):
     run_small(losa, wl, out_dtype=torch.bfloat16, in_fp32=False)
 
 
-def test_fp32_inputs_are_rounded_to_bf16(losa):
-    wl = W.custom("fp32in", 2, 64, (3, 10, 13), 64, amplitude=1.2, seed=11, in_dtype="fp32")
+TF32 = [
+    # name, heads, d, grid, block, text: the kind::tf32 kernels (d 128 runs
+    # 64-key stages, so a 128-token block spans two of them)
+    ("tf32_d64_b64", 2, 64, (3, 10, 13), 64, 0),
+    ("tf32_d64_b128_text", 2, 64, (2, 12, 20), 128, 30),
+    ("tf32_d64_b32", 2, 64, (3, 7, 9), 32, 0),
+    ("tf32_d128_b64", 2, 128, (3, 10, 13), 64, 0),
+    ("tf32_d128_b128_text", 2, 128, (2, 12, 20), 128, 30),
+    ("tf32_d128_b32", 2, 128, (3, 7, 9), 32, 5),
+]
+
+
+@pytest.mark.parametrize("name,heads,d,grid,block,text", TF32, ids=[s[0] for s in TF32])
+def test_fp32_inputs_take_the_tf32_path(losa, name, heads, d, grid, block, text):
+    wl = W.custom(name, heads, d, grid, block, text_tokens=text, amplitude=1.2,
+                  seed=zlib.crc32(name.encode()) % 1000, in_dtype="fp32")
     run_small(losa, wl, in_fp32=True)
+    run_small(losa, wl, in_fp32=True, out_dtype=torch.bfloat16, tau=0.95)
+
+
+def test_tf32_path_is_more_accurate_than_bf16_on_fp32_inputs(losa):
+    """On unrounded fp32 inputs, against fp64 on those same inputs: the fp32
+    (tf32) path's errors in the masses and in O are several times smaller
+    than those of the same inputs handed over as bf16."""
+    wl = W.custom("acc", 2, 128, (3, 10, 13), 64, amplitude=1.2, seed=13, in_dtype="fp32")
+    q, k, v = W.generate(wl, dtype=torch.float32)
+    L, b, scale = wl.seq_len, wl.block, 1 / math.sqrt(wl.head_dim)
+    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
+    o_ref, _ = O.dense_attention(q64, k64, v64, L, scale)
+    m_ref = O.block_mass(q64, k64, L, b, scale)
+    err = {}
+    for dt in (torch.float32, torch.bfloat16):
+        o, _, mass = losa.dense_mass(*(t.to("cuda", dt) for t in (q, k, v)), L, b)
+        torch.cuda.synchronize()
+        err[dt] = (np.abs(f64(mass) - m_ref).max(), np.abs(f64(o)[:, :, :L] - o_ref[:, :, :L]).max())
+    assert err[torch.float32][0] * 4 < err[torch.bfloat16][0], err
+    assert err[torch.float32][1] * 4 < err[torch.bfloat16][1], err
 
 
 def test_tau_one_keeps_every_positive_block_and_equals_dense(losa):

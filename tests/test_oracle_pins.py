@@ -315,17 +315,63 @@ def test_tiny_workload_prunes_in_band():
 
 
 def test_generator_is_seeded_and_bf16_exact():
-    wl = W.WORKLOADS["tiny"]
-    a = W.generate(wl)
-    b = W.generate(wl)
+    """bf16 workloads hand out bf16-exact values (any requested dtype); the
+    fp32 small workload hands out fp32 values that are not all bf16-exact."""
+    wl = W.custom("b16", 2, 64, (2, 8, 8), 32, amplitude=1.1, seed=4)
+    for dtype in (torch.float32, torch.float64):
+        for x in W.generate(wl, dtype=dtype):
+            assert x.dtype == dtype
+            assert torch.equal(x, x.to(torch.bfloat16).to(dtype))
+    tiny = W.WORKLOADS["tiny"]
+    a = W.generate(tiny)
+    b = W.generate(tiny)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
         assert x.dtype == torch.float32
-        assert torch.equal(x, x.to(torch.bfloat16).to(torch.float32))
-        assert torch.all(x[:, :, wl.seq_len:] == 0)
-    c = W.drift(wl, a, step=1)
+        assert not torch.equal(x, x.to(torch.bfloat16).to(torch.float32))
+        assert torch.all(x[:, :, tiny.seq_len:] == 0)
+    c = W.drift(tiny, a, step=1)
     assert not torch.equal(c[0], a[0])
     assert float((c[0] - a[0]).abs().max()) < 0.5
+
+
+def _tf32_exact(x):
+    """Round-to-nearest-even to 11 significant bits, in exact rationals."""
+    X = Fraction(float(x))
+    if X == 0:
+        return 0.0
+    e = math.floor(math.log2(abs(X)))
+    while Fraction(2) ** e > abs(X):
+        e -= 1
+    while Fraction(2) ** (e + 1) <= abs(X):
+        e += 1
+    ulp = Fraction(2) ** (max(e, -126) - 10)
+    return float(round(X / ulp) * ulp)  # round() on a Fraction: ties to even
+
+
+def test_round_tf32_matches_exact_rational_rounding():
+    """workloads.round_tf32 (the tf32 values the oracle is handed for fp32
+    inputs) against round-half-even in exact rationals: random values over
+    many binades, and every tie and near-tie pattern of the dropped bits."""
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(4000, generator=g) * torch.pow(2.0, torch.randint(-30, 30, (4000,),
+                                                                      generator=g).float())
+    base = torch.tensor([1.0, 1.5, -3.25, 1e-3, 7e5], dtype=torch.float32)
+    bits = base.view(torch.int32)
+    pats = []
+    for low in (0x0000, 0x0FFF, 0x1000, 0x1001, 0x1FFF, 0x0001, 0x17FF, 0x0800):
+        for odd in (0, 1):
+            pats.append(((bits & ~0x3FFF) | (odd << 13) | low).view(torch.float32))
+    x = torch.cat([x.float()] + pats)
+    r = W.round_tf32(x)
+    want = torch.tensor([_tf32_exact(v) for v in x.tolist()], dtype=torch.float64)
+    assert torch.equal(r.double(), want)
+    assert torch.all((r.view(torch.int32) & 0x1FFF) == 0)
+    # ties: half an ulp rounds to the even neighbour
+    one = torch.tensor([1 + 2 ** -11, 1 + 3 * 2 ** -11, -(1 + 2 ** -11)], dtype=torch.float32)
+    assert W.round_tf32(one).tolist() == [1.0, 1 + 2 ** -9, -1.0]
+    assert torch.equal(W.round_tf32(torch.tensor([float("inf"), 0.0])),
+                       torch.tensor([float("inf"), 0.0]))
 
 
 # ------------------------------------------------------------------ planted mistakes

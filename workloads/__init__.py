@@ -32,8 +32,11 @@ Recipe (all workloads):
     tau = 0.99, to prune about 40 % of blocks (the pages' figure, inside the
     30-50 % band the workloads state), and is never retuned.
   * Later denoising steps drift every tensor: X_s = X_{s-1} + 0.05 * N(0, 1).
-  * Values are drawn in fp32, then rounded once to bf16 (round to nearest
-    even); the bf16 values are what both sides consume.
+  * Values are drawn in fp32. For a workload whose caller hands bf16 to the
+    library they are rounded once to bf16 (round to nearest even), and the
+    bf16 values are what both sides consume. For an fp32 workload (the small
+    one) they stay fp32: the library rounds them to tf32 on entry, and the
+    oracle is handed round_tf32 of the same values.
 """
 from __future__ import annotations
 
@@ -125,9 +128,10 @@ def _positions(wl: Workload, device) -> torch.Tensor:
 def generate(wl: Workload, device="cpu", seed=None, amplitude=None, dtype=None):
     """Draw the construction-step Q, K, V of one layer.
 
-    Returns (q, k, v), each [B, H, L_pad, d] contiguous, in `dtype`
-    (default: float32 holding bf16-rounded values when wl.in_dtype == 'fp32',
-    else bfloat16). Rows >= L are zero.
+    Returns (q, k, v), each [B, H, L_pad, d] contiguous, in `dtype` (default:
+    float32 when wl.in_dtype == 'fp32', else bfloat16). Values are
+    bf16-rounded for bf16 workloads whatever `dtype` is, and left unrounded
+    for fp32 workloads unless `dtype` is bfloat16. Rows >= L are zero.
     """
     seed = wl.seed if seed is None else seed
     amplitude = wl.amplitude if amplitude is None else amplitude
@@ -179,10 +183,30 @@ def drift(wl: Workload, qkv, step: int, device="cpu", dtype=None):
 
 
 def _finish(wl, tensors, dtype):
-    rounded = [t.to(torch.bfloat16) for t in tensors]
     if dtype is None:
         dtype = torch.float32 if wl.in_dtype == "fp32" else torch.bfloat16
+    if wl.in_dtype == "fp32" and dtype != torch.bfloat16:
+        return tuple(t.to(dtype).contiguous() for t in tensors)
+    rounded = [t.to(torch.bfloat16) for t in tensors]
     return tuple(t.to(dtype).contiguous() for t in rounded)
+
+
+def round_tf32(x: torch.Tensor) -> torch.Tensor:
+    """The value a tf32 operand holds for each fp32 element: the nearest
+    number with 11 significant bits (10 stored), ties to even, returned as
+    float32. This is input preparation for the oracle (the values the
+    library's tf32 path computes on), done through frexp and an integer
+    rounding of the significand rather than on the bit pattern: with
+    x = m * 2^e and 1/2 <= |m| < 1, the result is round(m * 2^11) * 2^(e - 11)
+    (torch.round rounds half to even); below the normal range the spacing
+    stays that of the smallest normal exponent. NaN and Inf pass through."""
+    x64 = x.to(torch.float64)
+    m, e = torch.frexp(x64)
+    e = torch.clamp(e, min=-125)
+    m = x64 * torch.pow(2.0, (-e).to(torch.float64))
+    r = torch.round(m * 2048.0) * torch.pow(2.0, (e - 11).to(torch.float64))
+    r = torch.where(torch.isfinite(x64), r, x64)
+    return r.to(torch.float32)
 
 
 def sample_query_blocks(wl: Workload, per_head: int, seed: int = 12345):
