@@ -176,6 +176,7 @@ extern "C" {
 int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype, int B, int H,
                     int L, int L_pad, int d, int block, float scale, void* o, int out_dtype,
                     float* lse, float* mass, void* stream) {
+  NvtxRange nvtx_range("losa_dense_mass");
   if (!q || !k || !v || !o || !lse || !mass) return LOSA_ERR_ARG;
   if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LOSA_ERR_ARG;
   if (!valid_attn_shape(B, H, L, L_pad, d, block)) return LOSA_ERR_ARG;
@@ -196,6 +197,7 @@ int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype, i
 
 int losa_select(const float* mass, int B, int H, int n_blocks, int block, double tau,
                 losa_pattern** out, void* stream) {
+  NvtxRange nvtx_range("losa_select");
   if (out) *out = nullptr;
   if (!mass || !out) return LOSA_ERR_ARG;
   if (B < 1 || H < 1 || n_blocks < 1 || n_blocks > 2047) return LOSA_ERR_ARG;
@@ -228,6 +230,7 @@ int losa_pattern_info(const losa_pattern* p, losa_pattern_view* view) {
 int losa_pattern_export(const losa_pattern* p, int32_t* row_ptr, int32_t* col_idx,
                         int64_t* retained_fx, int64_t* total_fx, int32_t* tile_ptr,
                         int32_t* tile_entry, int32_t* tile_order, void* stream) {
+  NvtxRange nvtx_range("losa_pattern_export");
   if (!p) return LOSA_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t R = int64_t(p->B) * p->H * p->n_blocks;
@@ -253,6 +256,7 @@ int losa_pattern_export(const losa_pattern* p, int32_t* row_ptr, int32_t* col_id
 int losa_pattern_import(const int32_t* row_ptr, const int32_t* col_idx,
                         const int64_t* retained_fx, const int64_t* total_fx, int B, int H,
                         int n_blocks, int block, losa_pattern** out, void* stream) {
+  NvtxRange nvtx_range("losa_pattern_import");
   if (out) *out = nullptr;
   if (!row_ptr || !col_idx || !out) return LOSA_ERR_ARG;
   if (B < 1 || H < 1 || n_blocks < 1 || n_blocks > 2047) return LOSA_ERR_ARG;
@@ -268,6 +272,7 @@ int losa_pattern_import(const int32_t* row_ptr, const int32_t* col_idx,
 int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, int d, int L,
                      float scale, const losa_pattern* p, void* o, int out_dtype, float* lse,
                      void* stream) {
+  NvtxRange nvtx_range("losa_sparse_attn");
   if (!q || !k || !v || !o || !p) return LOSA_ERR_ARG;
   if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LOSA_ERR_ARG;
   const int L_pad = p->n_blocks * p->block;
@@ -292,6 +297,7 @@ int losa_sparse_attn(const void* q, const void* k, const void* v, int in_dtype, 
 
 void losa_free(losa_pattern* p) {
   if (!p) return;
+  NvtxRange nvtx_range("losa_free");
   int prev = 0;
   cudaGetDevice(&prev);
   cudaSetDevice(p->device);
@@ -302,6 +308,7 @@ void losa_free(losa_pattern* p) {
 }
 
 int losa_check_status(void* stream) {
+  NvtxRange nvtx_range("losa_check_status");
   int* w = device_status_word();
   if (!w) return LOSA_ERR_CUDA;
   int h = 0;

@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/losa.h"
 
@@ -27,6 +28,16 @@ struct losa_pattern {
 };
 
 namespace losa {
+
+// An NVTX range named after the C entry point for the call's duration, so a
+// profiler's timeline shows the library's calls around their kernels (no
+// cost when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // True when the current device is an sm_100 part (the only target built).
 bool is_sm100();

@@ -114,6 +114,20 @@ def check_selection(pat, mass_gpu, tau, check_tile_lists=True):
     return ref, ex
 
 
+class Guarded:
+    """An output buffer followed by a canary tail of 4,096 elements holding
+    a fixed value: a kernel that writes past the buffer's end changes it."""
+
+    def __init__(self, shape, dtype):
+        n = math.prod(shape)
+        self.buf = torch.full((n + 4096,), 12345.5, dtype=dtype, device="cuda")
+        self.out = self.buf[:n].view(shape)
+        self.tail0 = self.buf[n:].clone()
+
+    def check(self, what):
+        assert torch.equal(self.buf[self.out.numel():], self.tail0), f"{what} wrote past its end"
+
+
 def computed_on(t, in_fp32):
     """The values the library computes on for inputs t (fp32 on the host)."""
     return W.round_tf32(t) if in_fp32 else t.to(torch.bfloat16).to(torch.float32)
@@ -126,9 +140,15 @@ def run_small(losa, wl, tau=0.99, out_dtype=torch.float32, in_fp32=None):
     dt = torch.float32 if in_fp32 else torch.bfloat16
     qd, kd, vd = (t.to("cuda", dt) for t in (q, k, v))
     L, b, scale = wl.seq_len, wl.block, 1 / math.sqrt(wl.head_dim)
-    o, lse, mass = losa.dense_mass(qd, kd, vd, L, b, out_dtype=out_dtype)
+    B, H, Lp, d = qd.shape
+    g_o, g_lse, g_mass = (Guarded((B, H, Lp, d), out_dtype), Guarded((B, H, Lp), torch.float32),
+                          Guarded((B, H, wl.n_blocks, wl.n_blocks), torch.float32))
+    o, lse, mass = losa.dense_mass(qd, kd, vd, L, b, out_dtype=out_dtype, o=g_o.out,
+                                   lse=g_lse.out, mass=g_mass.out)
     torch.cuda.synchronize()
     losa.check_status()
+    for g, what in ((g_o, "dense O"), (g_lse, "dense lse"), (g_mass, "mass")):
+        g.check(what)
     q64, k64, v64 = (computed_on(t, in_fp32).double().numpy() for t in (q, k, v))
     o_ref, lse_ref = O.dense_attention(q64, k64, v64, L, scale)
     mass_ref = O.block_mass(q64, k64, L, b, scale)
@@ -148,9 +168,13 @@ def run_small(losa, wl, tau=0.99, out_dtype=torch.float32, in_fp32=None):
 
     q2, k2, v2 = W.drift(wl, (q, k, v), step=1, dtype=torch.float32)
     q2d, k2d, v2d = (t.to("cuda", dt) for t in (q2, k2, v2))
-    o2, lse2 = losa.sparse_attn(q2d, k2d, v2d, L, pat, out_dtype=out_dtype)
+    g_o2, g_lse2 = Guarded((B, H, Lp, d), out_dtype), Guarded((B, H, Lp), torch.float32)
+    o2, lse2 = losa.sparse_attn(q2d, k2d, v2d, L, pat, out_dtype=out_dtype, o=g_o2.out,
+                                lse=g_lse2.out)
     torch.cuda.synchronize()
     losa.check_status()
+    g_o2.check("sparse O")
+    g_lse2.check("sparse lse")
     o2_ref, lse2_ref = O.sparse_attention(*(computed_on(t, in_fp32).double().numpy()
                                             for t in (q2, k2, v2)), L, b, scale,
                                           ref["row_ptr"], ref["col_idx"])
