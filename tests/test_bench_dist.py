@@ -65,3 +65,14 @@ def test_max_over_ranks_gloo():
     out = mp.get_context("spawn").Manager().dict()
     mp.start_processes(_worker, args=(port, out), nprocs=2, start_method="spawn", join=True)
     assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_list_schedule_makespan():
+    """The in-order list scheduling the scheduler analysis simulates: each
+    job goes, in order, to the worker that becomes free first."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench._list_schedule([3, 3, 3, 3], 2) == 6
+    assert bench._list_schedule([5, 1, 1, 1, 1, 1], 2) == 5
+    assert bench._list_schedule([1, 1, 1, 1, 1, 5], 2) == 7   # a long job last sets the tail
+    assert bench._list_schedule([2.5], 4) == 2.5

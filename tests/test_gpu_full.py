@@ -148,3 +148,47 @@ def test_full_size_workload(losa, name):
     if Lp > L:
         assert torch.all(o[:, :, L:] == 0).item()
         assert torch.all(torch.isneginf(lse[:, :, L:])).item()
+
+
+@pytest.mark.parametrize("name", ["cogvideox", "wan2.1-1.3b"])
+def test_full_size_fp32_inputs_take_the_tf32_path(losa, name):
+    """The kind::tf32 kernels at full size: the layer's inputs drawn in fp32
+    and left unrounded, the library rounding them to tf32 on entry; the
+    oracle is handed the same tf32 values. Sampled query blocks of every
+    head: O within 1e-2 + 2^-8 |O|, lse within 1e-4, masses within 1e-5,
+    selection bit-exact on the GPU's masses, and the sparse step's O."""
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS[name], in_dtype="fp32")
+    L, b, d, n = wl.seq_len, wl.block, wl.head_dim, wl.n_blocks
+    scale = 1 / math.sqrt(d)
+    tau = 0.99
+    q, k, v = W.generate(wl, device="cuda", dtype=torch.float32)
+    o, lse, mass = losa.dense_mass(q, k, v, L, b, out_dtype=torch.bfloat16)
+    pat = losa.select(mass, b, tau)
+    q2, k2, v2 = W.drift(wl, (q, k, v), step=1, device="cuda", dtype=torch.float32)
+    o2, lse2 = losa.sparse_attn(q2, k2, v2, L, pat, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    losa.check_status()
+    ex = pat.export("cpu")
+    rp, mass_cpu = ex["row_ptr"].numpy(), mass.cpu().numpy()
+    err_d, err_s = ErrAcc(f"{name} fp32 dense O"), ErrAcc(f"{name} fp32 sparse O")
+    samples = W.sample_query_blocks(wl, 4, seed=5)
+    for (bb, h) in sorted({(x, y) for (x, y, _) in samples}):
+        qh, kh, vh = (W.round_tf32(t[bb, h].cpu()).double().numpy() for t in (q, k, v))
+        q2h, k2h, v2h = (W.round_tf32(t[bb, h].cpu()).double().numpy() for t in (q2, k2, v2))
+        for I in [I for (x, y, I) in samples if (x, y) == (bb, h)]:
+            rows = np.arange(I * b, min((I + 1) * b, L))
+            o_ref, lse_ref = O.attention_rows(qh[rows], kh[:L], vh[:L], scale)
+            err_d.add(_rows(o, bb, h, rows), o_ref)
+            assert np.max(np.abs(_rows(lse, bb, h, rows) - lse_ref)) <= LSE_ATOL
+            m_ref = O.block_mass_row(qh[None, None], kh[None, None], L, b, scale, 0, 0, I)
+            assert np.max(np.abs(mass_cpu[bb, h, I] - m_ref)) <= MASS_ATOL
+            r = (bb * wl.heads + h) * n + I
+            kept, C, S = O.select_row(O.to_fixed(mass_cpu[bb, h, I]).tolist(), tau)
+            assert ex["col_idx"][rp[r]:rp[r + 1]].tolist() == kept
+            keys = O.retained_keys(kept, b, L)
+            o2_ref, lse2_ref = O.attention_rows(q2h[rows], k2h[keys], v2h[keys], scale)
+            err_s.add(_rows(o2, bb, h, rows), o2_ref)
+            assert np.max(np.abs(_rows(lse2, bb, h, rows) - lse2_ref)) <= LSE_ATOL
+    err_d.check_mean()
+    err_s.check_mean()
