@@ -149,3 +149,38 @@ def test_pattern_import_accepts_a_valid_csr_up_to_the_device_check(losa):
     # Valid (diagonal plus one neighbour): passes the host checks, then the
     # device check reports that no sm_100 GPU is present.
     assert _import(losa, [0, 2, 4, 6, 7], [0, 1, 0, 1, 2, 3, 3]) == -6
+
+
+def test_process_settings_reject_values_out_of_range(losa):
+    """losa_set_wait_limit takes 0 (the default) to 2^33 SM cycles and
+    losa_set_sparse_schedule 0 or 1; anything else is refused on the host
+    and leaves the setting as it was."""
+    lib = losa.lib()
+    for bad in (-1, (1 << 33) + 1, -(1 << 40)):
+        assert lib.losa_set_wait_limit(bad) == -1
+    assert lib.losa_set_wait_limit(0) == 0
+    for bad in (-1, 2, 7):
+        assert lib.losa_set_sparse_schedule(bad) == -1
+    assert lib.losa_set_sparse_schedule(0) == 0
+    assert lib.losa_selftest_wait(0, None) == -1
+
+
+def test_select_noalloc_rejects_bad_arguments(losa):
+    """Host-side checks of the allocation-free selection, before any device
+    work: null buffers, sizes, tau, a negative capacity, and more rows than
+    its fixed scratch holds."""
+    lib = losa.lib()
+    call = lambda *a: lib.losa_select_noalloc(*a, None)
+    ok = (FAKE, 1, 2, 8, ctypes.c_double(0.99), FAKE, FAKE, ctypes.c_int64(16), FAKE, FAKE)
+    for i in (0, 5, 6, 8, 9):  # each pointer argument set to NULL
+        args = list(ok)
+        args[i] = None
+        assert call(*args) == -1
+    for B, H, n in ((0, 2, 8), (1, 0, 8), (1, 2, 0), (1, 2, 2048), (1, 40, 2047)):
+        assert call(FAKE, B, H, n, ctypes.c_double(0.99), FAKE, FAKE, ctypes.c_int64(16),
+                    FAKE, FAKE) == -1
+    for tau in (0.0, 1.5, float("nan")):
+        assert call(FAKE, 1, 2, 8, ctypes.c_double(tau), FAKE, FAKE, ctypes.c_int64(16),
+                    FAKE, FAKE) == -1
+    assert call(FAKE, 1, 2, 8, ctypes.c_double(0.99), FAKE, FAKE, ctypes.c_int64(-1),
+                FAKE, FAKE) == -1
