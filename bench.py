@@ -451,10 +451,8 @@ def _list_schedule(costs, workers):
 
 
 def sched_analysis(losa, wl, args, dev, tau=0.99):
-    """What a persistent tile scheduler recovers in the sparse kernel: the
-    kernel timed with one CTA per pair of tiles (hardware dispatch, before
-    and after) and with one persistent CTA per SM, beside an upper bound
-    from two measurements and one simulation:
+    """Upper bound of what a persistent tile scheduler could recover in the
+    sparse kernel, from two measurements and one simulation:
       * fixed cost: the same kernel on a pattern with one key block per row
         (the diagonal), i.e. every CTA's setup, Q load, pipeline fill,
         epilogue and teardown with almost no iterations, against the real
@@ -476,14 +474,6 @@ def sched_analysis(losa, wl, args, dev, tau=0.99):
     o = torch.empty(B, H, wl.seq_pad, d, device=dev, dtype=torch.bfloat16)
     t_full = _event_ms(lambda: losa.sparse_attn(*q1, L, pat, out_dtype=torch.bfloat16, o=o,
                                                 want_lse=False), n=5, warm=2)
-    try:
-        losa.set_sparse_schedule(True)
-        t_persistent = _event_ms(lambda: losa.sparse_attn(*q1, L, pat, out_dtype=torch.bfloat16,
-                                                          o=o, want_lse=False), n=5, warm=2)
-    finally:
-        losa.set_sparse_schedule(False)
-    t_full2 = _event_ms(lambda: losa.sparse_attn(*q1, L, pat, out_dtype=torch.bfloat16, o=o,
-                                                 want_lse=False), n=5, warm=2)
     R = B * H * n
     diag = losa.import_pattern(torch.arange(R + 1, dtype=torch.int32),
                                torch.arange(n, dtype=torch.int32).repeat(B * H), B, H, n, b,
@@ -500,10 +490,7 @@ def sched_analysis(losa, wl, args, dev, tau=0.99):
     hw = _list_schedule(pairs, sms)
     persistent = _list_schedule(n_it, 2 * sms)
     rec = {"analysis": "sched", "workload": wl.name, "sms": sms, "tiles": len(n_it),
-           "ctas": len(pairs), "sparse_ms": t_full, "sparse_ms_again": t_full2,
-           "sparse_ms_persistent": t_persistent,
-           "persistent_speedup": 0.5 * (t_full + t_full2) / t_persistent,
-           "diag_pattern_ms": t_diag,
+           "ctas": len(pairs), "sparse_ms": t_full, "diag_pattern_ms": t_diag,
            "fixed_cost_share": t_diag / t_full,
            "hw_dispatch_loss": hw / ideal - 1.0, "persistent_loss": persistent / ideal - 1.0,
            "persistent_gain_bound": (t_diag / t_full) + (hw - persistent) / hw}

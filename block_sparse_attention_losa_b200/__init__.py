@@ -29,8 +29,8 @@ STATUS = {0: "LOSA_OK", -1: "LOSA_ERR_ARG", -2: "LOSA_ERR_CUDA", -3: "LOSA_ERR_N
 # Every symbol include/losa.h declares.
 EXPORTS = ("losa_dense_mass", "losa_select", "losa_pattern_info", "losa_pattern_export",
            "losa_pattern_import", "losa_select_noalloc", "losa_sparse_attn", "losa_free",
-           "losa_check_status", "losa_selftest_wait", "losa_set_sparse_schedule",
-           "losa_set_wait_limit", "losa_exp2_eval", "losa_strerror", "losa_version")
+           "losa_check_status", "losa_selftest_wait", "losa_set_wait_limit", "losa_exp2_eval",
+           "losa_strerror", "losa_version")
 NOALLOC_MAX_ROWS = 65536  # LOSA_NOALLOC_MAX_ROWS
 
 
@@ -80,8 +80,6 @@ def _load():
     lib.losa_check_status.restype = i32
     lib.losa_selftest_wait.argtypes = [i64, vp]
     lib.losa_selftest_wait.restype = i32
-    lib.losa_set_sparse_schedule.argtypes = [i32]
-    lib.losa_set_sparse_schedule.restype = i32
     lib.losa_set_wait_limit.argtypes = [i64]
     lib.losa_set_wait_limit.restype = i32
     lib.losa_exp2_eval.argtypes = [vp, vp, i64, vp]
@@ -276,12 +274,6 @@ def exp2_eval(x, stream=None):
 def check_status(stream=None):
     """Synchronises the stream and raises if a kernel reported a timeout."""
     _check("losa_check_status", _lib.losa_check_status(_stream(stream)))
-
-
-def set_sparse_schedule(persistent: bool):
-    """Sparse kernel grid for later launches: one CTA per pair of tiles
-    (False, hardware dispatch) or one persistent CTA per SM (True)."""
-    _check("losa_set_sparse_schedule", _lib.losa_set_sparse_schedule(1 if persistent else 0))
 
 
 def set_wait_limit(cycles: int = 0):

@@ -332,12 +332,6 @@ int losa_selftest_wait(int64_t limit_cycles, void* stream) {
              : LOSA_ERR_CUDA;
 }
 
-int losa_set_sparse_schedule(int persistent) {
-  if (persistent != 0 && persistent != 1) return LOSA_ERR_ARG;
-  set_sparse_persistent(persistent == 1);
-  return LOSA_OK;
-}
-
 int losa_set_wait_limit(int64_t limit_cycles) {
   if (limit_cycles < 0 || limit_cycles > (int64_t(1) << 33)) return LOSA_ERR_ARG;
   set_wait_limit(limit_cycles);

@@ -20,13 +20,6 @@ void set_wait_limit(long long cycles) {
   g_wait_limit.store(cycles > 0 ? cycles : kWaitLimitCycles);
 }
 
-// Grid of the sparse kernel: one CTA per pair of tiles (the hardware
-// dispatches them in the count-sorted order), or one CTA per SM, each
-// sweeping every gridDim-th pair of the same order (persistent).
-std::atomic<int> g_sparse_persistent{0};
-
-void set_sparse_persistent(bool on) { g_sparse_persistent.store(on ? 1 : 0); }
-
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -243,17 +236,8 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, bool tf32
   p.wait_limit = g_wait_limit.load();
   const int BH = pat->B * pat->H;
   p.n_tiles = int(pat->n_tiles);
+  const dim3 grid(unsigned((pat->n_tiles + 1) / 2));  // two tiles per CTA
   if (pat->n_tiles == 0) return cudaSuccess;
-  const int64_t n_items = (pat->n_tiles + 1) / 2;  // two tiles per item
-  int64_t ctas = n_items;
-  if (g_sparse_persistent.load()) {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return cudaErrorInvalidDevice;
-    ctas = std::min<int64_t>(n_items, sms);
-  }
-  const dim3 grid(static_cast<unsigned>(ctas));
 #define LOSA_SPARSE_CASE(TF_, D_, BN_, NSK_, NSV_, BLK_)                                        \
   if (tf32 == TF_ && d == D_ && pat->block == BLK_)                                             \
     return out_bf16                                                                             \

@@ -66,8 +66,8 @@ struct AttnLayout {
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
   // q_full[2], k_full/k_empty[NSK], v_full/v_empty[NSV], s_full[2], s_free[2],
-  // p_full[2], o_full[2], red_bar[2][2], drain, q_free[2]
-  static constexpr int N_BARS = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 1 + 2;
+  // p_full[2], o_full[2], red_bar[2][2], drain
+  static constexpr int N_BARS = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem addr, abort flag
   static constexpr int OFF_RED = OFF_MISC + 16;          // float red[2 tiles][2][4 warps][4]
   static constexpr int BYTES = OFF_RED + 2 * 2 * 4 * 4 * 4;
@@ -144,7 +144,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* o_full = p_full + 2;       // [2] MMA -> softmax t: last PV_t done
   uint64_t* red_bar = o_full + 2;      // [2][2] softmax t: mass reduction
   uint64_t* drain_bar = red_bar + 4;   // MMA drain after an abort
-  uint64_t* q_free = drain_bar + 1;    // [2] MMA -> producer: Q_t smem free (next item)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
@@ -152,45 +151,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work items: per tile t, its head, query tile and key list. Dense:
-  // one item per CTA, the adjacent query tiles 2x, 2x + 1 of head y. Sparse:
-  // item i is the pair of tiles tile_order[2i], tile_order[2i + 1]; the CTA
-  // takes items blockIdx.x, blockIdx.x + gridDim.x, ... So a grid of one CTA
-  // per item is the hardware's in-order dispatch of the count-sorted order,
-  // and a grid of one CTA per SM is a persistent sweep of the same order
-  // that keeps TMEM, barriers and the K/V rings across items. Every role
-  // walks the same items and decodes them itself.
-  const int n_items = kDense ? 1 : (p.n_tiles + 1) / 2;
-  const int item0 = kDense ? 0 : int(blockIdx.x);
-  const int item_step = kDense ? 1 : int(gridDim.x);
+  // ---- work items: per tile t, its head, query tile and key list
   int bh[2], qt[2], e_begin[2] = {0, 0}, n_ent[2] = {0, 0}, n_it[2];
-  auto decode = [&](int item) {
-    if constexpr (kDense) {
-      bh[0] = bh[1] = blockIdx.y;
-      qt[0] = 2 * blockIdx.x;
-      qt[1] = 2 * blockIdx.x + 1;  // may lie past the head: rows read as 0, nothing stored
-      n_it[0] = n_it[1] = p.n_kv;
-    } else {
+  if constexpr (kDense) {
+    bh[0] = bh[1] = blockIdx.y;
+    qt[0] = 2 * blockIdx.x;
+    qt[1] = 2 * blockIdx.x + 1;  // may lie past the head: rows read as 0, nothing stored
+    n_it[0] = n_it[1] = p.n_kv;
+  } else {
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int idx = 2 * item + t;
-        if (idx < p.n_tiles) {
-          const int tile = p.tile_order[idx];
-          bh[t] = tile / p.n_qt;
-          qt[t] = tile - bh[t] * p.n_qt;
-          e_begin[t] = p.tile_ptr[tile];
-          n_ent[t] = p.tile_ptr[tile + 1] - e_begin[t];
-          n_it[t] = CPE * ((n_ent[t] + EPI - 1) / EPI);
-        } else {  // the last item of an odd tile count: slot 1 idle
-          bh[t] = 0;
-          qt[t] = 0;
-          e_begin[t] = 0;
-          n_ent[t] = 0;
-          n_it[t] = 0;
-        }
+    for (int t = 0; t < 2; ++t) {
+      const int idx = 2 * blockIdx.x + t;
+      if (idx < p.n_tiles) {
+        const int tile = p.tile_order[idx];
+        bh[t] = tile / p.n_qt;
+        qt[t] = tile - bh[t] * p.n_qt;
+        e_begin[t] = p.tile_ptr[tile];
+        n_ent[t] = p.tile_ptr[tile + 1] - e_begin[t];
+        n_it[t] = CPE * ((n_ent[t] + EPI - 1) / EPI);
+      } else {
+        bh[t] = 0;
+        qt[t] = 0;
+        n_it[t] = 0;
       }
     }
-  };
+  }
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -211,8 +196,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&v_empty[s], 1);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(&q_free[0], 1);
-    mbar_init(&q_free[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -231,8 +214,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(&q_full[t], Lay::Q_BYTES);
+#pragma unroll
+        for (int s = 0; s < N_SLABS; ++s)
+          tma_load_3d(sQ + t * Lay::Q_BYTES + s * (BM * 128), &tm_q, &q_full[t],
+                      s * SLAB_COLS, qt[t] * BM, bh[t]);
+      }
       int kc = 0, vc = 0;
-      int qn[2] = {0, 0};  // Q copies issued per tile slot (one per item)
       bool ok = true;
       // One stage = BN keys = EPI boxes of BOX rows, stacked in each slab.
       auto load_k = [&](const int (&key_row)[EPI], int head) -> bool {
@@ -261,25 +251,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ++vc;
         return true;
       };
-      for (int item = item0; ok && item < n_items; item += item_step) {
-      decode(item);
-      // Q of both slots; from the second item on, once the previous item's
-      // last S MMA of that slot has read the old Q.
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (!ok) break;
-        if (qn[t] > 0 && !mbar_wait(&q_free[t], (qn[t] - 1) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&q_full[t], Lay::Q_BYTES);
-#pragma unroll
-        for (int s = 0; s < N_SLABS; ++s)
-          tma_load_3d(sQ + t * Lay::Q_BYTES + s * (BM * 128), &tm_q, &q_full[t],
-                      s * SLAB_COLS, qt[t] * BM, bh[t]);
-        ++qn[t];
-      }
-      if (!ok) break;
       if constexpr (kDense) {
         for (int j = 0; ok && j < p.n_kv; ++j) {
           const int rows[EPI] = {j * BN};
@@ -311,18 +282,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      }  // items
-      // Let the last Q copy of each slot land before the CTA exits (a slot
-      // with no work in the last item of an odd tile count has nobody else
-      // waiting for it; the others have landed already).
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-        if (qn[t] > 0) mbar_wait_drain(&q_full[t], (qn[t] - 1) & 1);
       if (!ok) {
-        // Aborted: wait (bounded) for the K/V copies still in flight before
-        // the CTA releases its shared memory.
+        // Aborted: wait (bounded) for the copies still in flight before the
+        // CTA releases its shared memory.
+        mbar_wait_drain(&q_full[0], 0);
+        mbar_wait_drain(&q_full[1], 0);
         for (int i = (kc > NSK ? kc - NSK : 0); i < kc; ++i) mbar_wait_drain(&k_full[i % NSK], (i / NSK) & 1);
         for (int i = (vc > NSV ? vc - NSV : 0); i < vc; ++i) mbar_wait_drain(&v_full[i % NSV], (i / NSV) & 1);
+      } else {
+        // A tile slot with no work (the last CTA of an odd tile count):
+        // nobody else waits for its Q copy, so let it land before exit.
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (n_it[t] == 0) mbar_wait_drain(&q_full[t], 0);
       }
     }
   } else if (warp == 9) {
@@ -332,16 +304,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t k_base = smem_addr(sK);
       const uint32_t v_base = smem_addr(sV);
       int kc = 0, vc = 0;
-      int pc[2] = {0, 0};  // P_t consumed (pass 1), over all items
-      int pv[2] = {0, 0};  // P_t V products of the current item
+      int pc[2] = {0, 0};  // P_t consumed (pass 1)
       int fc[2] = {0, 0};  // S_t uses in pass 2
-      int li = 0;          // items done
       bool ok = true;
       bool q_ready[2] = {false, false};
       // S_t = Q_t K^T into S_t's TMEM columns, from K stage ks.
       auto issue_s = [&](int t, int ks) -> bool {
         if (!q_ready[t]) {
-          if (!mbar_wait(&q_full[t], li & 1, wc)) return false;
+          if (!mbar_wait(&q_full[t], 0, wc)) return false;
           q_ready[t] = true;
         }
         tc_fence_after();
@@ -384,13 +354,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t vaddr = v_base + vs * Lay::KV_BYTES + kk * (K_STEP * 128);
           if constexpr (kTf32)
             umma_tf32_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128_32b(vaddr, BN * 128, 512), IDESC_PV,
-                         (pv[t] > 0 || kk > 0) ? 1u : 0u);
+                         (pc[t] > 0 || kk > 0) ? 1u : 0u);
           else
             umma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(vaddr, BN * 128, 1024), IDESC_PV,
-                         (pv[t] > 0 || kk > 0) ? 1u : 0u);
+                         (pc[t] > 0 || kk > 0) ? 1u : 0u);
         }
         ++pc[t];
-        ++pv[t];
         return true;
       };
       auto wait_v = [&](int& vs) -> bool {
@@ -402,10 +371,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ++vc;
       };
 
-      for (int item = item0; ok && item < n_items; item += item_step, ++li) {
-      decode(item);
-      q_ready[0] = q_ready[1] = false;
-      pv[0] = pv[1] = 0;
       if constexpr (kDense) {
         const int n = p.n_kv;
         int ks, vs;
@@ -443,19 +408,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           release_k(ks);
         }
       } else {
-        // q_free[t] fires when the item's last S_t MMA (the last reader of
-        // Q_t) completes, so the producer can bring the next item's Q_t in
-        // while this item's last P.V products and softmax still run.
         int ks, vs;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!ok) break;
-          if (n_it[t] > 0) {
+          if (ok && n_it[t] > 0) {
             ok = wait_k(ks) && issue_s(t, ks);
-            if (!ok) break;
-            release_k(ks);
+            if (ok) release_k(ks);
           }
-          if (n_it[t] <= 1) umma_commit(&q_free[t]);
         }
         const int n_max = max(n_it[0], n_it[1]);
         for (int j = 0; ok && j < n_max; ++j) {
@@ -469,14 +428,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               ok = wait_k(ks) && issue_s(t, ks);
               if (!ok) break;
               release_k(ks);
-              if (j + 2 == n_it[t]) umma_commit(&q_free[t]);
             } else {
               umma_commit(&o_full[t]);
             }
           }
         }
       }
-      }  // items
       if (!ok) {
         // Drain: let every MMA issued so far finish before TMEM is freed.
         umma_commit(drain_bar);
@@ -490,17 +447,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int t = warp >> 2;               // query tile of this warpgroup
     const int wl = warp & 3;               // warp within the warpgroup
     const int r = wl * 32 + lane;          // row within the tile, TMEM lane
+    const int row = qt[t] * BM + r;        // token row within the head
     const uint32_t lane_base = uint32_t(wl * 32) << 16;
     const uint32_t s_col = tmem + lane_base + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
     const uint32_t o_col = tmem + lane_base + (t ? Lay::TMEM_O1 : Lay::TMEM_O0);
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    int sc = 0;              // S_t completions seen (all items)
-    int oc = 0;              // O_t completions seen (items with work in this slot)
-    bool ok = true;
-    for (int item = item0; ok && item < n_items; item += item_step) {
-    decode(item);
-    const int row = qt[t] * BM + r;        // token row within the head
     const int n_iter = n_it[t];
     const int n = kDense ? n_iter : n_ent[t];  // list entries (sparse)
     // Running row max in log2 units. It is raised as soon as a tile exceeds
@@ -514,6 +466,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // and the tile sums are accumulated with Kahan compensation (a plain
     // running sum loses the small terms against the large total).
     float l = 0.f, l_c = 0.f;
+    int sc = 0;              // S_t completions seen
+    bool ok = true;
 
     // List entries run one iteration ahead: those of iteration j + 1 are
     // fetched at the top of iteration j, so their global-load latency hides
@@ -680,8 +634,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const bool row_valid = row < p.L && n_iter > 0;
     const float lse2 = (l > 0.f) ? m_used + log2f(l) : __int_as_float(0x7f800000);
     if (ok && n_iter > 0) {
-      if (!mbar_wait(&o_full[t], oc & 1, wc)) ok = false;
-      ++oc;
+      if (!mbar_wait(&o_full[t], 0, wc)) ok = false;
       tc_fence_after();
     }
     if (ok && n_iter > 0) {
@@ -837,7 +790,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-    }  // items
   }
 
   tc_fence_before();

@@ -70,10 +70,6 @@ cudaError_t launch_sparse(const void* q, const void* k, const void* v, bool tf32
 // 0 restores the default.
 void set_wait_limit(long long cycles);
 
-// Sparse kernel grid: one CTA per pair of tiles (false, hardware dispatch)
-// or one persistent CTA per SM (true), for launches after the call.
-void set_sparse_persistent(bool on);
-
 // One bounded mbarrier wait that must run out (diagnostic).
 cudaError_t launch_wait_selftest(long long limit_cycles, cudaStream_t stream);
 

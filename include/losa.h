@@ -46,8 +46,7 @@
  *     word (set by a kernel that ran out of a bounded wait, or by a bad mass
  *     value), one stream-ordered memory pool (patterns and scratch), the
  *     fixed scratch array of losa_select_noalloc, and its CUDA function
- *     handles; and, per process, the wait limit of losa_set_wait_limit and
- *     the sparse schedule of losa_set_sparse_schedule.
+ *     handles; and, per process, the wait limit of losa_set_wait_limit.
  *     Calls on different streams are independent, except that overlapping
  *     losa_select_noalloc calls share that scratch array.
  */
@@ -273,20 +272,6 @@ void losa_free(losa_pattern* p);
  * or LOSA_ERR_CUDA. The word records the first event only.
  */
 int losa_check_status(void* stream);
-
-/*
- * losa_set_sparse_schedule - how losa_sparse_attn launches its tiles (for
- * the whole process, launches after the call). The pattern orders the
- * 128-row tiles head by head and, within a head, by entry count, largest
- * first; the kernel takes them two at a time. persistent = 0: one CTA per
- * pair of tiles, which the hardware dispatches in that order (the default);
- * persistent = 1: one CTA per SM, each sweeping every (number of SMs)-th
- * pair of the same order and keeping its tensor memory, barriers and K/V
- * rings across pairs, loading the next pair's Q while the current one
- * finishes. Results are bit-identical either way. Not for use while other
- * threads launch. Returns LOSA_ERR_ARG for any other value.
- */
-int losa_set_sparse_schedule(int persistent);
 
 /*
  * losa_set_wait_limit - diagnostic of the attention kernels' failure path:

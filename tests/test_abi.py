@@ -152,16 +152,12 @@ def test_pattern_import_accepts_a_valid_csr_up_to_the_device_check(losa):
 
 
 def test_process_settings_reject_values_out_of_range(losa):
-    """losa_set_wait_limit takes 0 (the default) to 2^33 SM cycles and
-    losa_set_sparse_schedule 0 or 1; anything else is refused on the host
-    and leaves the setting as it was."""
+    """losa_set_wait_limit takes 0 (the default) to 2^33 SM cycles; anything
+    else is refused on the host and leaves the setting as it was."""
     lib = losa.lib()
     for bad in (-1, (1 << 33) + 1, -(1 << 40)):
         assert lib.losa_set_wait_limit(bad) == -1
     assert lib.losa_set_wait_limit(0) == 0
-    for bad in (-1, 2, 7):
-        assert lib.losa_set_sparse_schedule(bad) == -1
-    assert lib.losa_set_sparse_schedule(0) == 0
     assert lib.losa_selftest_wait(0, None) == -1
 
 

@@ -380,44 +380,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(losa):
     assert torch.allclose(mass.sum(-1), torch.ones_like(mass.sum(-1)), atol=1e-4)
 
 
-PERSIST = [
-    # name, heads, d, grid, block, in_fp32: more pairs of tiles than SMs, so
-    # each persistent CTA walks several; the last case has an odd tile count
-    # (101 heads x 3 tiles), so one item has an idle slot.
-    ("bf16_d128_b64", 40, 128, (4, 16, 16), 64, False),
-    ("bf16_d64_b128", 40, 64, (4, 16, 16), 128, False),
-    ("bf16_d128_b32_odd", 101, 128, (2, 12, 16), 32, False),
-    ("tf32_d128_b128", 40, 128, (4, 16, 16), 128, True),
-]
-
-
-@pytest.mark.parametrize("name,heads,d,grid,block,in_fp32", PERSIST, ids=[c[0] for c in PERSIST])
-def test_persistent_schedule_is_bit_identical(losa, name, heads, d, grid, block, in_fp32):
-    """The same tiles swept by one persistent CTA per SM (TMEM, barriers and
-    K/V rings kept across pairs of tiles, the next pair's Q loaded early)
-    give bit for bit what the hardware's dispatch of one CTA per pair gives."""
-    wl = W.custom(name, heads, d, grid, block, amplitude=1.2, seed=51)
-    dt = torch.float32 if in_fp32 else torch.bfloat16
-    q, k, v = (t.to("cuda", dt) for t in W.generate(wl, dtype=torch.float32))
-    L = wl.seq_len
-    _, _, mass = losa.dense_mass(q, k, v, L, block)
-    pat = losa.select(mass, block, 0.95)
-    assert (pat.n_tiles + 1) // 2 > torch.cuda.get_device_properties(0).multi_processor_count
-    o_hw, lse_hw = losa.sparse_attn(q, k, v, L, pat)
-    try:
-        losa.set_sparse_schedule(True)
-        o_p, lse_p = losa.sparse_attn(q, k, v, L, pat)
-        o_pb, _ = losa.sparse_attn(q, k, v, L, pat, out_dtype=torch.bfloat16)
-    finally:
-        losa.set_sparse_schedule(False)
-    o_hb, _ = losa.sparse_attn(q, k, v, L, pat, out_dtype=torch.bfloat16)
-    torch.cuda.synchronize()
-    losa.check_status()
-    assert torch.equal(o_hw, o_p) and torch.equal(lse_hw, lse_p) and torch.equal(o_hb, o_pb)
-
-
-@pytest.mark.parametrize("persistent", [False, True])
-def test_attention_kernels_abort_on_a_short_wait_limit(losa, persistent):
+def test_attention_kernels_abort_on_a_short_wait_limit(losa):
     """The attention kernels' own failure path: with a wait limit of one SM
     cycle, the first wait of the construction and of the sparse kernel that
     is not satisfied at once gives up; the call reports LOSA_ERR_TIMEOUT
@@ -436,7 +399,6 @@ def test_attention_kernels_abort_on_a_short_wait_limit(losa, persistent):
     losa.check_status()
     assert lib.losa_set_wait_limit(-1) == -1
     try:
-        losa.set_sparse_schedule(persistent)
         losa.set_wait_limit(1)
         losa.dense_mass(q, k, v, L, b)
         with pytest.raises(losa.LosaError) as e:
@@ -448,7 +410,6 @@ def test_attention_kernels_abort_on_a_short_wait_limit(losa, persistent):
         assert e.value.status == -4
     finally:
         losa.set_wait_limit(0)               # back to the default
-        losa.set_sparse_schedule(False)
     o, lse, mass = losa.dense_mass(q, k, v, L, b)
     o2, lse2 = losa.sparse_attn(q, k, v, L, pat)
     torch.cuda.synchronize()
