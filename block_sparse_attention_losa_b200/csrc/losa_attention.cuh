@@ -66,8 +66,9 @@ struct AttnLayout {
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
   // q_full[2], k_full/k_empty[NSK], v_full/v_empty[NSV], s_full[2], s_free[2],
-  // p_full[2], o_full[2], red_bar[2][2], drain
-  static constexpr int N_BARS = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 1;
+  // p_full[2], o_full[2], red_bar[2][2], drain; then, for the double-buffered
+  // mass pass, s2_full[2][2], s2_free[2][2], o_read[2]
+  static constexpr int N_BARS = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 1 + 10;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem addr, abort flag
   static constexpr int OFF_RED = OFF_MISC + 16;          // float red[2 tiles][2][4 warps][4]
   static constexpr int BYTES = OFF_RED + 2 * 2 * 4 * 4 * 4;
@@ -76,6 +77,12 @@ struct AttnLayout {
   static constexpr int SMEM_ALLOC = BYTES + 1024 > 120 * 1024 ? BYTES + 1024 : 120 * 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
+  // Second S buffer of each tile in the construction kernel's mass pass,
+  // where O is dead (stored by the epilogue): at D = 128 O_t's own columns;
+  // at D = 64 the unused columns [384, 512) for tile 0 and both O regions
+  // [256, 384) for tile 1.
+  static constexpr int TMEM_ALT0 = D == 128 ? 256 : 384;
+  static constexpr int TMEM_ALT1 = D == 128 ? 384 : 256;
   static_assert(D % 64 == 0 && D <= 128, "head dim must be 64 or 128");
   static_assert(BN % 32 == 0 && BN <= 128, "key tile must be 32, 64 or 128");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "1 KB alignment");
@@ -121,6 +128,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int CPE = BLK > BN ? BLK / BN : 1;  // key stages per list entry / key block
   constexpr int K_STEP = 32 / ESZ;         // K of one MMA instruction (32 bytes of a row)
   static_assert((BN % BLK == 0 || BLK % BN == 0) && BLK % 32 == 0, "block size");
+  // The construction kernel's mass pass double-buffers S (the second buffer
+  // in columns O no longer needs) at b = 128, where that measured faster;
+  // at b = 32 and 64 the single buffer measured faster.
+  constexpr bool kDblMass = kDense && BLK == 128;
   constexpr uint32_t IDESC_S = kTf32 ? idesc_tf32_f32(BM, BN, false, false)
                                      : idesc_bf16_f32(BM, BN, false, false);
   constexpr uint32_t IDESC_PV = kTf32 ? idesc_tf32_f32(BM, D, false, true)
@@ -144,6 +155,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* o_full = p_full + 2;       // [2] MMA -> softmax t: last PV_t done
   uint64_t* red_bar = o_full + 2;      // [2][2] softmax t: mass reduction
   uint64_t* drain_bar = red_bar + 4;   // MMA drain after an abort
+  uint64_t* s2_full = drain_bar + 1;   // [2][2] MMA -> softmax t: S_t buffer ready (kDblMass)
+  uint64_t* s2_free = s2_full + 4;     // [2][2] softmax t -> MMA: S_t buffer read (kDblMass)
+  uint64_t* o_read = s2_free + 4;      // [2] softmax t -> MMA: O_t read (kDblMass)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
@@ -196,6 +210,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&v_empty[s], 1);
     }
     mbar_init(drain_bar, 1);
+    if (kDblMass) {
+      for (int i = 0; i < 4; ++i) {
+        mbar_init(&s2_full[i], 1);
+        mbar_init(&s2_free[i], 128);
+      }
+      mbar_init(&o_read[0], 128);
+      mbar_init(&o_read[1], 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -308,15 +330,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int fc[2] = {0, 0};  // S_t uses in pass 2
       bool ok = true;
       bool q_ready[2] = {false, false};
-      // S_t = Q_t K^T into S_t's TMEM columns, from K stage ks.
-      auto issue_s = [&](int t, int ks) -> bool {
+      // S_t = Q_t K^T into TMEM columns col (S_t's own by default), from K
+      // stage ks; `done` (s_full[t] by default) is committed when it completes.
+      auto issue_s = [&](int t, int ks, int col = -1, uint64_t* done = nullptr) -> bool {
         if (!q_ready[t]) {
           if (!mbar_wait(&q_full[t], 0, wc)) return false;
           q_ready[t] = true;
         }
         tc_fence_after();
         const uint32_t qb = q_base + t * Lay::Q_BYTES;
-        const uint32_t d_tmem = tmem + (t ? Lay::TMEM_S1 : Lay::TMEM_S0);
+        const uint32_t d_tmem = tmem + (col >= 0 ? col : (t ? Lay::TMEM_S1 : Lay::TMEM_S0));
         // 32 bytes of K per instruction: four steps per 128-byte slab.
 #pragma unroll
         for (int kk = 0; kk < D / K_STEP; ++kk) {
@@ -328,7 +351,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           else
             umma_bf16_ss(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[t]);
+        umma_commit(done ? done : &s_full[t]);
         return true;
       };
       auto wait_k = [&](int& ks) -> bool {
@@ -395,17 +418,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             umma_commit(&o_full[1]);
           }
         }
-        // ---- pass 2: S only; S_t is free again once softmax t has read it
-        for (int j = 0; ok && j < n; ++j) {
-          if (!(ok = wait_k(ks))) break;
+        if constexpr (kDblMass) {
+          // ---- pass 2, double-buffered: S_t(j) goes to buffer j & 1 (S_t's
+          // own columns, or the second buffer, free once the epilogue has
+          // read the O columns it overlaps), so S_t(j + 1) is computed while
+          // softmax t sums S_t(j). A buffer is reused once softmax t has read
+          // the S it held two key tiles before.
+          for (int j = 0; ok && j < n; ++j) {
+            if (!(ok = wait_k(ks))) break;
+            const int bsel = j & 1;
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (ok && fc[t] > 0) ok = mbar_wait(&s_free[t], (fc[t] - 1) & 1, wc);
-            if (ok) ok = issue_s(t, ks);
-            ++fc[t];
+            for (int t = 0; t < 2; ++t) {
+              if (ok && j >= 2) ok = mbar_wait(&s2_free[2 * t + bsel], ((j >> 1) - 1) & 1, wc);
+              if (ok && j == 1) {
+                if constexpr (D == 128) {
+                  ok = mbar_wait(&o_read[t], 0, wc);
+                } else if (t == 1) {
+                  ok = mbar_wait(&o_read[0], 0, wc) && mbar_wait(&o_read[1], 0, wc);
+                }
+              }
+              if (ok)
+                ok = issue_s(t, ks, bsel ? (t ? Lay::TMEM_ALT1 : Lay::TMEM_ALT0)
+                                         : (t ? Lay::TMEM_S1 : Lay::TMEM_S0),
+                             &s2_full[2 * t + bsel]);
+            }
+            if (!ok) break;
+            release_k(ks);
           }
-          if (!ok) break;
-          release_k(ks);
+        } else {
+          // ---- pass 2: S only; S_t is free again once softmax t has read it
+          for (int j = 0; ok && j < n; ++j) {
+            if (!(ok = wait_k(ks))) break;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (ok && fc[t] > 0) ok = mbar_wait(&s_free[t], (fc[t] - 1) & 1, wc);
+              if (ok) ok = issue_s(t, ks);
+              ++fc[t];
+            }
+            if (!ok) break;
+            release_k(ks);
+          }
         }
       } else {
         int ks, vs;
@@ -670,6 +722,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (row_in && p.lse != nullptr)
         p.lse[size_t(bh[t]) * p.L_pad + row] =
             (row_valid && l > 0.f) ? lse2 * 0.69314718055994531f : NEG_INF;
+      if constexpr (kDblMass) {
+        // O_t is stored: its columns may take pass 2's second S buffer.
+        tc_fence_before();
+        mbar_arrive(&o_read[t]);
+      }
     }
 
     if constexpr (kDense) {
@@ -684,17 +741,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float lsub = row_valid ? lse2 : __int_as_float(0x7f800000);
       float* red_t = red + t * 32;
       float carry = 0.f;  // a key block over CPE key tiles: the earlier tiles' sum
+      // kDblMass: S_t(j) sits in buffer j & 1, S_t's own columns or the
+      // second buffer.
+      const uint32_t alt_col = tmem + lane_base + (t ? Lay::TMEM_ALT1 : Lay::TMEM_ALT0);
       for (int j = 0; ok && j < n_iter; ++j) {
-        if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
-        ++sc;
-        tc_fence_after();
         float s[BN];
+        if constexpr (kDblMass) {
+          const int bsel = j & 1;
+          if (!mbar_wait(&s2_full[2 * t + bsel], (j >> 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t src = bsel ? alt_col : s_col;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-          tmem_ld32(s_col + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&s_free[t]);
+          for (int c = 0; c < BN / 32; ++c)
+            tmem_ld32(src + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&s2_free[2 * t + bsel]);
+        } else {
+          if (!mbar_wait(&s_full[t], sc & 1, wc)) { ok = false; break; }
+          ++sc;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+            tmem_ld32(s_col + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&s_free[t]);
+        }
 
         const int key0 = j * BN;
         // Padded query rows subtract +inf (their scores are finite: rows past
