@@ -61,6 +61,8 @@ def parse_args():
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the fused construction + selection comparison")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small profiling cases)")
     ap.add_argument("--ncu-case", action="store_true",
@@ -88,11 +90,12 @@ def load_peaks():
 
 
 def attention_source_sha():
-    """Hash of the attention kernel's code: the two sources with // comments,
-    trailing blanks and empty lines removed (a comment edit keeps the hash)."""
+    """Hash of the attention kernel's code: its three sources with //
+    comments, trailing blanks and empty lines removed (a comment edit keeps
+    the hash)."""
     import hashlib
     h = hashlib.sha256()
-    for f in ("losa_attention.cuh", "losa_device.cuh"):
+    for f in ("losa_attention.cuh", "losa_device.cuh", "losa_cut.cuh"):
         with open(os.path.join(ROOT, "block_sparse_attention_losa_b200", "csrc", f)) as fh:
             for line in fh:
                 code = line.split("//", 1)[0].rstrip()
@@ -674,6 +677,8 @@ def main():
         "clocks": clock_info,
     }
 
+    if not args.no_fused:
+        line["fused_select"] = fused_select_measure(losa, qkv0, L, b, tau, o_dense, lse, mass)
     if not args.no_e2e:
         line["e2e"] = e2e_measure(losa, wl, qkv0, distinct, n_sparse, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -688,6 +693,34 @@ def main():
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def fused_select_measure(losa, qkv0, L, b, tau, o, lse, mass, n=3):
+    """Construction + selection as one call (the cut fused into the
+    construction kernel's epilogue) against the two separate calls, on the
+    step's construction inputs, outside the timed step: CUDA-event ms of
+    each (both include the selection's one host synchronisation), and
+    whether the two patterns' CSR and tile lists are bit-identical."""
+    def separate():
+        losa.dense_mass(*qkv0, L, b, out_dtype=torch.bfloat16, o=o, lse=lse, mass=mass)
+        losa.select(mass, b, tau).close()
+
+    def fused():
+        losa.dense_mass_select(*qkv0, L, b, tau=tau, out_dtype=torch.bfloat16, o=o, lse=lse,
+                               mass=mass)[3].close()
+
+    sep_ms = _event_ms(separate, n=n, warm=1)
+    fused_ms = _event_ms(fused, n=n, warm=1)
+    losa.dense_mass(*qkv0, L, b, out_dtype=torch.bfloat16, o=o, lse=lse, mass=mass)
+    p1 = losa.select(mass, b, tau)
+    p2 = losa.dense_mass_select(*qkv0, L, b, tau=tau, out_dtype=torch.bfloat16)[3]
+    e1, e2 = p1.export("cpu"), p2.export("cpu")
+    # tile_order is unique only up to ties, so it is left out
+    same = all(torch.equal(e1[k], e2[k]) for k in e1 if k != "tile_order")
+    p1.close()
+    p2.close()
+    losa.check_status()
+    return {"ms": fused_ms, "separate_ms": sep_ms, "csr_and_tiles_bit_identical": same}
 
 
 def e2e_measure(losa, wl, qkv0, distinct, n_sparse, args, world, max_host_sets=4):

@@ -27,7 +27,8 @@ STATUS = {0: "LOSA_OK", -1: "LOSA_ERR_ARG", -2: "LOSA_ERR_CUDA", -3: "LOSA_ERR_N
           -4: "LOSA_ERR_TIMEOUT", -5: "LOSA_ERR_MASS", -6: "LOSA_ERR_UNSUPPORTED"}
 
 # Every symbol include/losa.h declares.
-EXPORTS = ("losa_dense_mass", "losa_select", "losa_pattern_info", "losa_pattern_export",
+EXPORTS = ("losa_dense_mass", "losa_select", "losa_dense_mass_select", "losa_pattern_info",
+           "losa_pattern_export",
            "losa_pattern_import", "losa_select_noalloc", "losa_sparse_attn", "losa_free",
            "losa_check_status", "losa_selftest_wait", "losa_set_wait_limit", "losa_exp2_eval",
            "losa_strerror", "losa_version")
@@ -62,6 +63,9 @@ def _load():
     lib.losa_dense_mass.restype = i32
     lib.losa_select.argtypes = [vp, i32, i32, i32, i32, f64, ctypes.POINTER(vp), vp]
     lib.losa_select.restype = i32
+    lib.losa_dense_mass_select.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32,
+                                           f64, vp, i32, vp, vp, ctypes.POINTER(vp), vp]
+    lib.losa_dense_mass_select.restype = i32
     lib.losa_pattern_info.argtypes = [vp, ctypes.POINTER(PatternView)]
     lib.losa_pattern_info.restype = i32
     lib.losa_pattern_export.argtypes = [vp] * 9
@@ -215,6 +219,31 @@ def select(mass, block, tau=0.99, stream=None):
                           _stream(stream))
     _check("losa_select", st)
     return Pattern(h, mass.device)
+
+
+def dense_mass_select(q, k, v, L, block, tau=0.99, scale=None, out_dtype=torch.float32,
+                      o=None, lse=None, mass=None, stream=None):
+    """Construction and selection in one call, the per-row cut fused into
+    the construction kernel: (o, lse, mass, Pattern), each as dense_mass and
+    select would give them."""
+    _check_qkv(q, k, v)
+    B, H, Lp, d = q.shape
+    n = Lp // block
+    scale = default_scale(d) if scale is None else scale
+    dev = q.device
+    if o is None:
+        o = torch.empty(B, H, Lp, d, device=dev, dtype=out_dtype)
+    if lse is None:
+        lse = torch.empty(B, H, Lp, device=dev, dtype=torch.float32)
+    if mass is None:
+        mass = torch.empty(B, H, n, n, device=dev, dtype=torch.float32)
+    h = ctypes.c_void_p()
+    st = _lib.losa_dense_mass_select(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q),
+                                     B, H, int(L), Lp, d, int(block), float(scale), float(tau),
+                                     o.data_ptr(), _dtype_code(o), lse.data_ptr(),
+                                     mass.data_ptr(), ctypes.byref(h), _stream(stream))
+    _check("losa_dense_mass_select", st)
+    return o, lse, mass, Pattern(h, dev)
 
 
 def import_pattern(row_ptr, col_idx, B, H, n_blocks, block, retained_fx=None, total_fx=None,

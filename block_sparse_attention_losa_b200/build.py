@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblosa.so")
 SOURCES = ["losa_api.cu", "losa_attention.cu", "losa_select.cu"]
-HEADERS = ["losa_device.cuh", "losa_attention.cuh", "losa_internal.h"]
+HEADERS = ["losa_device.cuh", "losa_attention.cuh", "losa_cut.cuh", "losa_internal.h"]
 
 
 def nvcc_path() -> str:

@@ -195,6 +195,36 @@ int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype, i
   return LOSA_OK;
 }
 
+int losa_dense_mass_select(const void* q, const void* k, const void* v, int in_dtype, int B,
+                           int H, int L, int L_pad, int d, int block, float scale, double tau,
+                           void* o, int out_dtype, float* lse, float* mass, losa_pattern** out,
+                           void* stream) {
+  NvtxRange nvtx_range("losa_dense_mass_select");
+  if (out) *out = nullptr;
+  if (!q || !k || !v || !o || !lse || !mass || !out) return LOSA_ERR_ARG;
+  if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LOSA_ERR_ARG;
+  if (!valid_attn_shape(B, H, L, L_pad, d, block)) return LOSA_ERR_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return LOSA_ERR_ARG;
+  if (!(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_ARG;
+  if (!is_sm100()) return LOSA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  KernelInputs in;
+  in.s = s;
+  const int64_t n_elem = int64_t(B) * H * L_pad * d;
+  int st = prepare_inputs(in, q, k, v, in_dtype, n_elem);
+  if (st != LOSA_OK) return st;
+  SelectJob job;
+  st = select_begin(B, H, L_pad / block, block, tau, s, job);
+  if (st != LOSA_OK) return st;
+  if (launch_dense(in.q, in.k, in.v, in.tf32, B * H, L, L_pad, d, block, scale, o,
+                   out_dtype == LOSA_BF16, lse, mass, s, &job.cut) != cudaSuccess) {
+    select_abort(job);
+    return LOSA_ERR_CUDA;
+  }
+  return select_end(mass, /*run_cut=*/false, job, out);
+}
+
 int losa_select(const float* mass, int B, int H, int n_blocks, int block, double tau,
                 losa_pattern** out, void* stream) {
   NvtxRange nvtx_range("losa_select");

@@ -57,12 +57,13 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int L_pad, int d, int 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK, bool kTf32>
+template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK, bool kTf32,
+          bool kCut = false>
 cudaError_t run(const void* q, const void* k, const void* v, int BH, AttnParams p,
                 dim3 grid, cudaStream_t stream) {
   constexpr int ESZ = kTf32 ? 4 : 2;
   using Lay = AttnLayout<D, BN, NSK, NSV, ESZ>;
-  auto kern = attn_kernel<D, BN, NSK, NSV, kDense, kOutBf16, BLK, kTf32>;
+  auto kern = attn_kernel<D, BN, NSK, NSV, kDense, kOutBf16, BLK, kTf32, kCut>;
   // Cheap, and per device: set on every launch.
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM_ALLOC);
@@ -173,7 +174,7 @@ cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStrea
 
 cudaError_t launch_dense(const void* q, const void* k, const void* v, bool tf32, int BH, int L,
                          int L_pad, int d, int block, float scale, void* o, bool out_bf16,
-                         float* lse, float* mass, cudaStream_t stream) {
+                         float* lse, float* mass, cudaStream_t stream, const CutOutputs* cut) {
   AttnParams p{};
   p.L = L;
   p.L_pad = L_pad;
@@ -185,6 +186,13 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, bool tf32,
   p.o = o;
   p.lse = lse;
   p.mass = mass;
+  if (cut) {
+    p.tau_fx = cut->tau_fx;
+    p.cut_key = cut->cut_key;
+    p.cut_count = cut->count;
+    p.retained_fx = cut->retained_fx;
+    p.total_fx = cut->total_fx;
+  }
   p.status = device_status_word();
   if (!p.status) return cudaErrorInvalidDevice;
   p.wait_limit = g_wait_limit.load();
@@ -193,11 +201,18 @@ cudaError_t launch_dense(const void* q, const void* k, const void* v, bool tf32,
 // stages of 128 keys (32 KB each); bf16 d 64: 32 KB + 4 + 4 stages of 16 KB;
 // tf32 d 64: 64 KB + 3 + 2 stages of 32 KB; tf32 d 128: 128 KB + 2 K + 1 V
 // stage of 64 keys (32 KB each).
-#define LOSA_DENSE_CASE(TF_, D_, BN_, NSK_, NSV_, BLK_)                                        \
-  if (tf32 == TF_ && d == D_ && block == BLK_)                                                 \
-    return out_bf16                                                                            \
-               ? run<D_, BN_, NSK_, NSV_, true, true, BLK_, TF_>(q, k, v, BH, p, grid, stream) \
-               : run<D_, BN_, NSK_, NSV_, true, false, BLK_, TF_>(q, k, v, BH, p, grid, stream);
+// With a cut, the kCut instance (same kernel plus the fused selection cut).
+#define LOSA_DENSE_CASE(TF_, D_, BN_, NSK_, NSV_, BLK_)                                          \
+  if (tf32 == TF_ && d == D_ && block == BLK_) {                                                 \
+    if (cut)                                                                                     \
+      return out_bf16 ? run<D_, BN_, NSK_, NSV_, true, true, BLK_, TF_, true>(q, k, v, BH, p,    \
+                                                                              grid, stream)      \
+                      : run<D_, BN_, NSK_, NSV_, true, false, BLK_, TF_, true>(q, k, v, BH, p,   \
+                                                                               grid, stream);    \
+    return out_bf16                                                                              \
+               ? run<D_, BN_, NSK_, NSV_, true, true, BLK_, TF_>(q, k, v, BH, p, grid, stream)   \
+               : run<D_, BN_, NSK_, NSV_, true, false, BLK_, TF_>(q, k, v, BH, p, grid, stream); \
+  }
   LOSA_DENSE_CASE(false, 128, 128, 3, 2, 128)
   LOSA_DENSE_CASE(false, 128, 128, 3, 2, 64)
   LOSA_DENSE_CASE(false, 128, 128, 3, 2, 32)

@@ -30,6 +30,7 @@
 // post, Phase 3 - Repeated Sparse Inference).
 #pragma once
 
+#include "losa_cut.cuh"
 #include "losa_device.cuh"
 
 namespace losa {
@@ -51,6 +52,14 @@ struct AttnParams {
   const int* tile_order;  // sparse only
   int* status;
   long long wait_limit;   // SM cycles a wait spins before it gives up
+  // Fused selection cut (the construction kernel's kCut instances): per
+  // mass row the cut key, kept count and fixed-point sums of the threshold
+  // tau_fx = round(tau * 2^48), as losa_select's cut computes them.
+  unsigned long long tau_fx;
+  unsigned long long* cut_key;
+  int* cut_count;
+  long long* retained_fx;
+  long long* total_fx;
 };
 
 // ESZ: bytes per operand element (2 = bf16, 4 = fp32 read as tf32). Every
@@ -98,6 +107,11 @@ struct AttnLayout {
 template <int D> constexpr int poly_pairs_flash() { return 0; }
 template <int D> constexpr int poly_pairs_mass() { return 7; }
 
+// Workspace of one warpgroup's fused selection cut, at the start of the
+// (by then free) operand staging memory.
+constexpr int kCutSmemStride = 32768;
+static_assert(sizeof(cut::BucketSmem) <= kCutSmemStride, "cut workspace");
+
 constexpr int kAttnThreads = 384;
 constexpr int kAttnLaunchRegs = 168;   // checked against ptxas at build time
 constexpr int kSoftmaxRegs = 216;
@@ -114,7 +128,8 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kAttnThreads * kAtt
 // takes CPE = b / BN iterations.
 // kTf32: Q, K, V are fp32 (already rounded to tf32) and every MMA is
 // kind::tf32; the weights P stay fp32 in TMEM as the tf32 A operand of P V.
-template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK, bool kTf32>
+template <int D, int BN, int NSK, int NSV, bool kDense, bool kOutBf16, int BLK, bool kTf32,
+          bool kCut = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -132,6 +147,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // in columns O no longer needs) at b = 128, where that measured faster;
   // at b = 32 and 64 the single buffer measured faster.
   constexpr bool kDblMass = kDense && BLK == 128;
+  static_assert(!kCut || (kDense && 2 * kCutSmemStride <= Lay::OFF_BAR),
+                "the fused cut runs in the construction kernel, in its staging memory");
   constexpr uint32_t IDESC_S = kTf32 ? idesc_tf32_f32(BM, BN, false, false)
                                      : idesc_bf16_f32(BM, BN, false, false);
   constexpr uint32_t IDESC_PV = kTf32 ? idesc_tf32_f32(BM, D, false, true)
@@ -859,6 +876,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int w = 0; w < WPB; ++w) tot += rb[(wl + w) * 4 + kb];
               if (J0 + kb < p.n_blocks) mrow[J0 + kb] = tot * inv_cnt;
             }
+          }
+        }
+      }
+
+      if constexpr (kCut) {
+        // Fused selection: this CTA holds every key block of its query
+        // blocks' mass rows, so each warpgroup cuts its own tile's rows here.
+        // Once both tiles' mass passes are over, every MMA has read its
+        // operands (each S was waited for), so the Q/K/V staging memory is
+        // free for the cut's workspace, and the barrier makes the mass rows
+        // these warps wrote visible to them. A warp that gave up a wait, or
+        // an abort anywhere in the CTA, skips the cut in both warpgroups.
+        __syncwarp();
+        __threadfence_block();
+        const bool quit = named_bar_or(1, 256, !ok || *abort_flag != 0);
+        if (!quit) {
+          auto& sm = *reinterpret_cast<cut::BucketSmem*>(smem + t * kCutSmemStride);
+          const WarpgroupSync wg_sync{2 + t};
+          for (int q = 0; q < BM / BLK; ++q) {
+            const int I = qt[t] * (BM / BLK) + q;
+            if (I >= p.n_blocks) break;
+            const int64_t mr = int64_t(bh[t]) * p.n_blocks + I;
+            cut::bucket_cut_row<128>(p.mass + mr * p.n_blocks, p.n_blocks, p.tau_fx, sm, r,
+                                     wg_sync, mr, p.cut_key, p.cut_count, p.retained_fx,
+                                     p.total_fx, p.status);
           }
         }
       }

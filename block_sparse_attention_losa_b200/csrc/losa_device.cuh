@@ -278,6 +278,28 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Named barrier `id` (1..15; 0 is __syncthreads) over `count` threads
+// (whole warps), with the memory ordering of a CTA barrier among them.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// The same barrier, returning whether `pred` held in any of the threads.
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+// A barrier functor over one warpgroup (128 threads) on named barrier `id`.
+struct WarpgroupSync {
+  int id;
+  __device__ __forceinline__ void operator()() const { named_bar_sync(id, 128); }
+};
+
 // Per-warpgroup register budget (all four warps of a warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void reg_alloc() {

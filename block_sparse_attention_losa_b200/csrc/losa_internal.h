@@ -53,12 +53,24 @@ cudaMemPool_t device_pool();
 // Stream-ordered allocation from device_pool(); nullptr on failure.
 void* pool_alloc(size_t bytes, cudaStream_t stream);
 
+// Per-row outputs of the selection's threshold cut (device arrays of R =
+// B*H*n entries) and the fixed-point threshold round(tau * 2^48).
+struct CutOutputs {
+  unsigned long long tau_fx;
+  unsigned long long* cut_key;
+  int* count;
+  long long* retained_fx;
+  long long* total_fx;
+};
+
 // Runs the dense two-pass construction kernel. q/k/v are bf16 device
 // pointers, or fp32 ones already rounded to tf32 when tf32 is set; the
-// arguments were validated by the caller.
+// arguments were validated by the caller. With `cut`, the kernel also runs
+// the selection's cut on every mass row it wrote (the fused path).
 cudaError_t launch_dense(const void* q, const void* k, const void* v, bool tf32, int BH, int L,
                          int L_pad, int d, int block, float scale, void* o, bool out_bf16,
-                         float* lse, float* mass, cudaStream_t stream);
+                         float* lse, float* mass, cudaStream_t stream,
+                         const CutOutputs* cut = nullptr);
 
 // Runs the block-sparse kernel over pattern p (validated by the caller);
 // q/k/v as for launch_dense.
@@ -87,6 +99,30 @@ cudaError_t launch_f32_to_tf32(const float* src, float* dst, int64_t n, cudaStre
 // Returns a losa_status.
 int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
                   losa_pattern** out, cudaStream_t stream);
+
+// build_pattern in two halves, so that the construction kernel can run the
+// per-row cut itself (losa_dense_mass_select): select_begin allocates the
+// pattern and its scratch and exposes the cut's output arrays in `cut`;
+// select_end runs the cut (unless it already ran), the tile lists and the
+// tile order, synchronises once for the CSR size and completes the pattern.
+// Both return a losa_status; on failure everything is released.
+struct SelectJob {
+  losa_pattern* p = nullptr;
+  char* fixed = nullptr;
+  char* scratch = nullptr;
+  CutOutputs cut{};
+  int* tcnt = nullptr;
+  int* hist = nullptr;
+  int* cursor = nullptr;
+  int64_t R = 0, T = 0, n_keys = 0;
+  int n = 0, n_qt = 0, qpt = 0;
+  unsigned long long tau_fx = 0;
+  cudaStream_t stream = nullptr;
+};
+int select_begin(int B, int H, int n, int block, double tau, cudaStream_t stream,
+                 SelectJob& job);
+int select_end(const float* mass, bool run_cut, SelectJob& job, losa_pattern** out);
+void select_abort(SelectJob& job);
 
 // Builds a pattern from a host CSR that the caller has validated (row_ptr
 // monotone from 0 with non-empty rows, columns strictly ascending in

@@ -19,36 +19,20 @@
 #include <mutex>
 #include <vector>
 
+#include "losa_cut.cuh"
 #include "losa_device.cuh"
 #include "losa_internal.h"
 
 namespace losa {
 namespace {
 
+using cut::kNoKey;
+using cut::kXMax;
+using cut::reaches;
+using cut::sort_key;
+using cut::to_fixed;
+
 constexpr int kSelThreads = 256;
-constexpr unsigned long long kXMax = (1ull << 49) - 1;          // masses in [0, 2); J < 2048
-constexpr unsigned long long kNoKey = ~0ull;
-
-// x = round(m * 2^48) (ties to even; exact, as m * 2^48 only shifts the
-// exponent). Returns false for NaN, Inf, negative or >= 2.
-__device__ __forceinline__ bool to_fixed(float m, long long& x) {
-  if (!(m >= 0.f && m < 2.f)) {
-    x = 0;
-    return false;
-  }
-  x = __double2ll_rn(double(m) * 281474976710656.0);
-  return true;
-}
-
-__device__ __forceinline__ unsigned long long sort_key(long long x, int J) {
-  return ((kXMax - (unsigned long long)x) << 11) | (unsigned long long)J;
-}
-
-// 2^48 * C >= tau_fx * S, exactly.
-__device__ __forceinline__ bool reaches(unsigned long long C, unsigned long long tau_fx,
-                                        unsigned long long S) {
-  return ((unsigned __int128)C << 48) >= (unsigned __int128)tau_fx * S;
-}
 
 // One warp per row: the cut key, kept count, kept and total fixed-point
 // mass. The row's NP sort keys (n rounded up to a power of two, padded with
@@ -178,186 +162,25 @@ __global__ void __launch_bounds__(32 * kCutWarps)
   }
 }
 
-// Rows of more than 512 key blocks: one CTA per row. The keys are bucketed
-// by the leading five bits of x (the highest set bit and the four below it: 16 buckets per
-// octave of mass, x = 0 in bucket 0), so every key of a higher bucket has a
-// larger x than every key of a lower one. The bucket in which the running sum
-// over buckets in descending order first reaches the threshold is found with
-// a block scan, and only that bucket's keys are sorted (bitonic, in shared
-// memory): the keys of the buckets above fill the first positions of the
-// sorted order whatever their own order, so the cut (position, key and
-// prefix sum) is the one the full sort-and-accumulate definition gives.
-// Bucket sums and counts are integer atomics: the result does not depend on
-// scheduling.
+// Rows of more than 512 key blocks: one CTA of 256 threads per row, running
+// the bucketed cut of losa_cut.cuh (the construction kernel's fused epilogue
+// runs the same code on a warpgroup).
 constexpr int kBkThreads = 256;
-constexpr int kBkPerThread = 4;
-constexpr int kBuckets = 1 + 49 * 16;  // x < 2^49
-constexpr int kBkCap = 2048;           // n <= 2047 keys, padded to a power of two
-static_assert(kBkThreads * kBkPerThread >= kBuckets, "bucket scan coverage");
+constexpr int kBkCap = cut::kCap;
 
-__device__ __forceinline__ int x_bucket(unsigned long long x) {
-  if (x == 0) return 0;
-  const int h = 63 - __clzll((long long)x);
-  const int sub = h >= 4 ? int((x >> (h - 4)) & 15u) : int((x << (4 - h)) & 15u);
-  return 1 + h * 16 + sub;
-}
+struct CtaSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
 
 __global__ void __launch_bounds__(kBkThreads)
     select_cut_bucket_kernel(const float* __restrict__ mass, int n, unsigned long long tau_fx,
                              unsigned long long* __restrict__ cut_key, int* __restrict__ count,
                              long long* __restrict__ retained_fx, long long* __restrict__ total_fx,
                              int* status) {
-  using ScanU = cub::BlockScan<unsigned long long, kBkThreads>;
-  using ScanI = cub::BlockScan<int, kBkThreads>;
-  using Reduce = cub::BlockReduce<int, kBkThreads>;
-  __shared__ unsigned long long hsum[kBuckets];
-  __shared__ int hcnt[kBuckets];
-  __shared__ unsigned long long cand[kBkCap];
-  __shared__ union {
-    typename ScanU::TempStorage scan_u;
-    typename ScanI::TempStorage scan_i;
-    typename Reduce::TempStorage reduce;
-  } tmp;
-  __shared__ unsigned long long sh_A, sh_S;
-  __shared__ int sh_b, sh_above, sh_m, sh_k;
-  const int t = threadIdx.x;
+  __shared__ cut::BucketSmem sm;
   const int64_t row = blockIdx.x;
-  const float* mrow = mass + size_t(row) * n;
-
-  for (int i = t; i < kBuckets; i += kBkThreads) {
-    hsum[i] = 0;
-    hcnt[i] = 0;
-  }
-  if (t == 0) sh_m = 0;
-  __syncthreads();
-  bool bad = false;
-  for (int J = t; J < n; J += kBkThreads) {
-    long long x;
-    bad |= !to_fixed(mrow[J], x);
-    const int b = x_bucket((unsigned long long)x);
-    atomicAdd(&hsum[b], (unsigned long long)x);
-    atomicAdd(&hcnt[b], 1);
-  }
-  if (__any_sync(0xffffffffu, bad) && (t & 31) == 0) atomicCAS(status, kStatusOk, kStatusBadMass);
-  __syncthreads();
-
-  // Buckets in descending order: thread t owns reversed positions
-  // [t * 4, t * 4 + 4), i.e. buckets kBuckets - 1 - pos.
-  unsigned long long ls = 0;
-  int lc = 0;
-#pragma unroll
-  for (int i = 0; i < kBkPerThread; ++i) {
-    const int pos = t * kBkPerThread + i;
-    if (pos < kBuckets) {
-      ls += hsum[kBuckets - 1 - pos];
-      lc += hcnt[kBuckets - 1 - pos];
-    }
-  }
-  unsigned long long sum_before, S;
-  ScanU(tmp.scan_u).ExclusiveSum(ls, sum_before, S);
-  __syncthreads();
-  int cnt_before;
-  ScanI(tmp.scan_i).ExclusiveSum(lc, cnt_before);
-  __syncthreads();
-  // First bucket (in descending order) whose inclusive sum reaches the
-  // threshold; an all-zero row (S = 0) stops at its first key, in bucket 0.
-  int first = kBuckets;
-  unsigned long long A_at = 0;
-  int above_at = 0;
-  {
-    unsigned long long A = sum_before;
-    int above = cnt_before;
-#pragma unroll
-    for (int i = 0; i < kBkPerThread; ++i) {
-      const int pos = t * kBkPerThread + i;
-      if (pos >= kBuckets || first != kBuckets) break;
-      const int b = kBuckets - 1 - pos;
-      if (S > 0 ? reaches(A + hsum[b], tau_fx, S) : b == 0) {
-        first = pos;
-        A_at = A;
-        above_at = above;
-      }
-      A += hsum[b];
-      above += hcnt[b];
-    }
-  }
-  const int pmin = Reduce(tmp.reduce).Reduce(first, cub::Min());
-  if (t == 0) sh_k = pmin;
-  __syncthreads();
-  if (first == sh_k && first < kBuckets) {
-    sh_b = kBuckets - 1 - first;
-    sh_A = A_at;
-    sh_above = above_at;
-    sh_S = S;
-  }
-  __syncthreads();
-  const int bstar = sh_b;
-  // The boundary bucket's keys (the row is in L1 by now).
-  for (int J = t; J < n; J += kBkThreads) {
-    long long x;
-    to_fixed(mrow[J], x);
-    if (x_bucket((unsigned long long)x) == bstar) cand[atomicAdd(&sh_m, 1)] = sort_key(x, J);
-  }
-  __syncthreads();
-  const int m = sh_m;
-  int np = 2;
-  while (np < m) np <<= 1;
-  for (int i = m + t; i < np; i += kBkThreads) cand[i] = kNoKey;
-  // Bitonic sort of the bucket, ascending.
-  for (int size = 2; size <= np; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int pr = t; pr < np / 2; pr += kBkThreads) {
-        const int i = 2 * stride * (pr / stride) + (pr % stride);
-        const int k = i + stride;
-        const unsigned long long a = cand[i], b = cand[k];
-        const bool up = (i & size) == 0;
-        if ((a > b) == up) {
-          cand[i] = b;
-          cand[k] = a;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  // Prefix sums over the sorted bucket, on top of the buckets above it:
-  // thread t owns positions [t * per, t * per + per).
-  const int per = (np + kBkThreads - 1) / kBkThreads;
-  auto xval = [](unsigned long long key) -> unsigned long long {
-    return key == kNoKey ? 0ull : kXMax - (key >> 11);
-  };
-  unsigned long long local = 0;
-  for (int i = 0; i < per; ++i) {
-    const int pos = t * per + i;
-    if (pos < m) local += xval(cand[pos]);
-  }
-  unsigned long long before;
-  ScanU(tmp.scan_u).ExclusiveSum(local, before);
-  __syncthreads();
-  const unsigned long long St = sh_S;
-  unsigned long long C = sh_A + before;
-  int firstk = kBkCap;
-  for (int i = 0; i < per; ++i) {
-    const int pos = t * per + i;
-    if (pos >= m) break;
-    C += xval(cand[pos]);
-    if (reaches(C, tau_fx, St)) {
-      firstk = pos;
-      break;
-    }
-  }
-  const int kmin = Reduce(tmp.reduce).Reduce(firstk, cub::Min());
-  if (t == 0) sh_k = kmin;
-  __syncthreads();
-  const int p = sh_k;
-  if (p < m && p >= t * per && p < t * per + per) {
-    // The thread that owns the cut position writes the row's results; its
-    // running sum C stopped exactly there.
-    cut_key[row] = cand[p];
-    count[row] = sh_above + p + 1;
-    retained_fx[row] = (long long)C;
-    total_fx[row] = (long long)St;
-  }
+  cut::bucket_cut_row<kBkThreads>(mass + size_t(row) * n, n, tau_fx, sm, int(threadIdx.x),
+                                  CtaSync{}, row, cut_key, count, retained_fx, total_fx, status);
 }
 
 // Launches the cut kernel with the smallest power-of-two capacity >= n.
@@ -550,27 +373,30 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
-                  losa_pattern** out, cudaStream_t stream) {
+int select_begin(int B, int H, int n, int block, double tau, cudaStream_t stream,
+                 SelectJob& job) {
+  job = SelectJob{};
   const int BH = B * H;
-  const int64_t R = int64_t(BH) * n;
+  job.R = int64_t(BH) * n;
   const int L_pad = n * block;
-  const int n_qt = (L_pad + 127) / 128;
-  const int qpt = 128 / block;
-  const int64_t T = int64_t(BH) * n_qt;
-  const unsigned long long tau_fx = (unsigned long long)llrint(tau * 281474976710656.0);
-  int* status = device_status_word();
-  if (!status) return LOSA_ERR_CUDA;
+  job.n = n;
+  job.n_qt = (L_pad + 127) / 128;
+  job.qpt = 128 / block;
+  job.T = int64_t(BH) * job.n_qt;
+  job.tau_fx = (unsigned long long)llrint(tau * 281474976710656.0);
+  job.stream = stream;
+  const int64_t R = job.R, T = job.T;
 
   losa_pattern* p = new losa_pattern{};
   p->B = B;
   p->H = H;
   p->n_blocks = n;
   p->block = block;
-  p->n_qt = n_qt;
+  p->n_qt = job.n_qt;
   p->n_tiles = T;
   p->stream = stream;
   cudaGetDevice(&p->device);
+  job.p = p;
 
   // Pattern arrays of known size: one allocation.
   const size_t o_row = 0;
@@ -583,46 +409,74 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
   const size_t s_cut = 0;
   const size_t s_cnt = s_cut + align256(R * 8);
   const size_t s_tcnt = s_cnt + align256(R * 4);
-  const int64_t n_keys = int64_t(BH) * (n + 1);  // order keys: head x (n + 1)
+  job.n_keys = int64_t(BH) * (n + 1);  // order keys: head x (n + 1)
   const size_t s_hist = s_tcnt + align256(T * 4);
-  const size_t s_cur = s_hist + align256(n_keys * 4);
-  const size_t scratch_bytes = s_cur + align256((n_keys + 1) * 4);
+  const size_t s_cur = s_hist + align256(job.n_keys * 4);
+  const size_t scratch_bytes = s_cur + align256((job.n_keys + 1) * 4);
 
-  char* fixed = static_cast<char*>(pool_alloc(fixed_bytes, stream));
-  char* scratch = static_cast<char*>(pool_alloc(scratch_bytes, stream));
+  job.fixed = static_cast<char*>(pool_alloc(fixed_bytes, stream));
+  job.scratch = static_cast<char*>(pool_alloc(scratch_bytes, stream));
+  if (!job.fixed || !job.scratch) {
+    select_abort(job);
+    return LOSA_ERR_NOMEM;
+  }
+  p->fixed_mem = job.fixed;
+  p->row_ptr = reinterpret_cast<int32_t*>(job.fixed + o_row);
+  p->tile_ptr = reinterpret_cast<int32_t*>(job.fixed + o_tptr);
+  p->tile_order = reinterpret_cast<int32_t*>(job.fixed + o_tord);
+  p->retained_fx = reinterpret_cast<int64_t*>(job.fixed + o_ret);
+  p->total_fx = reinterpret_cast<int64_t*>(job.fixed + o_tot);
+  job.cut.tau_fx = job.tau_fx;
+  job.cut.cut_key = reinterpret_cast<unsigned long long*>(job.scratch + s_cut);
+  job.cut.count = reinterpret_cast<int*>(job.scratch + s_cnt);
+  job.cut.retained_fx = reinterpret_cast<long long*>(p->retained_fx);
+  job.cut.total_fx = reinterpret_cast<long long*>(p->total_fx);
+  job.tcnt = reinterpret_cast<int*>(job.scratch + s_tcnt);
+  job.hist = reinterpret_cast<int*>(job.scratch + s_hist);
+  job.cursor = reinterpret_cast<int*>(job.scratch + s_cur);
+  return LOSA_OK;
+}
+
+void select_abort(SelectJob& job) {
+  if (job.fixed) cudaFreeAsync(job.fixed, job.stream);
+  if (job.scratch) cudaFreeAsync(job.scratch, job.stream);
+  if (job.p && job.p->list_mem) cudaFreeAsync(job.p->list_mem, job.stream);
+  delete job.p;
+  job = SelectJob{};
+}
+
+int select_end(const float* mass, bool run_cut, SelectJob& job, losa_pattern** out) {
+  losa_pattern* p = job.p;
+  cudaStream_t stream = job.stream;
+  const int64_t R = job.R, T = job.T;
+  const int n = job.n, qpt = job.qpt, n_qt = job.n_qt;
+  int* status = device_status_word();
+  if (!status) {
+    select_abort(job);
+    return LOSA_ERR_CUDA;
+  }
   auto fail = [&](int code) {
-    if (fixed) cudaFreeAsync(fixed, stream);
-    if (scratch) cudaFreeAsync(scratch, stream);
-    if (p->list_mem) cudaFreeAsync(p->list_mem, stream);
-    delete p;
+    select_abort(job);
     return code;
   };
-  if (!fixed || !scratch) return fail(LOSA_ERR_NOMEM);
-  p->fixed_mem = fixed;
-  p->row_ptr = reinterpret_cast<int32_t*>(fixed + o_row);
-  p->tile_ptr = reinterpret_cast<int32_t*>(fixed + o_tptr);
-  p->tile_order = reinterpret_cast<int32_t*>(fixed + o_tord);
-  p->retained_fx = reinterpret_cast<int64_t*>(fixed + o_ret);
-  p->total_fx = reinterpret_cast<int64_t*>(fixed + o_tot);
-  auto* cut = reinterpret_cast<unsigned long long*>(scratch + s_cut);
-  auto* cnt = reinterpret_cast<int*>(scratch + s_cnt);
-  auto* tcnt = reinterpret_cast<int*>(scratch + s_tcnt);
-  auto* hist = reinterpret_cast<int*>(scratch + s_hist);
-  auto* cursor = reinterpret_cast<int*>(scratch + s_cur);
-
-  launch_select_cut(mass, R, n, tau_fx, cut, cnt, (long long*)p->retained_fx,
-                    (long long*)p->total_fx, status, stream);
-  tile_count_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(mass, cut, n, qpt, n_qt, tcnt);
+  unsigned long long* cut = job.cut.cut_key;
+  int* cnt = job.cut.count;
+  if (run_cut)
+    launch_select_cut(mass, R, n, job.tau_fx, cut, cnt, job.cut.retained_fx, job.cut.total_fx,
+                      status, stream);
+  tile_count_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(mass, cut, n, qpt, n_qt, job.tcnt);
   scan_kernel<<<1, 1024, 0, stream>>>(cnt, int(R), p->row_ptr);
-  scan_kernel<<<1, 1024, 0, stream>>>(tcnt, int(T), p->tile_ptr);
-  cudaMemsetAsync(hist, 0, n_keys * sizeof(int), stream);
+  scan_kernel<<<1, 1024, 0, stream>>>(job.tcnt, int(T), p->tile_ptr);
+  cudaMemsetAsync(job.hist, 0, job.n_keys * sizeof(int), stream);
   const int og = int(std::min<int64_t>((T + 255) / 256, 1024));
-  order_hist_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n_qt, n, hist);
-  scan_kernel<<<1, 1024, 0, stream>>>(hist, int(n_keys), cursor);
-  order_scatter_kernel<<<og, 256, 0, stream>>>(tcnt, int(T), n_qt, n, cursor, p->tile_order);
+  order_hist_kernel<<<og, 256, 0, stream>>>(job.tcnt, int(T), n_qt, n, job.hist);
+  scan_kernel<<<1, 1024, 0, stream>>>(job.hist, int(job.n_keys), job.cursor);
+  order_scatter_kernel<<<og, 256, 0, stream>>>(job.tcnt, int(T), n_qt, n, job.cursor,
+                                               p->tile_order);
   if (cudaGetLastError() != cudaSuccess) return fail(LOSA_ERR_CUDA);
 
-  // The one host synchronisation: CSR sizes and the mass check.
+  // The one host synchronisation: CSR sizes and the status word (a bad mass
+  // value, or a wait a fused construction kernel gave up).
   int totals[2] = {0, 0};
   int host_status = 0;
   if (cudaMemcpyAsync(&totals[0], p->row_ptr + R, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
@@ -648,13 +502,19 @@ int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
   p->tile_entry = reinterpret_cast<int32_t*>(lists + align256(size_t(p->nnz) * 4));
   tile_write_kernel<<<unsigned(T), kSelThreads, 0, stream>>>(
       mass, cut, n, qpt, n_qt, p->row_ptr, p->tile_ptr, p->col_idx, p->tile_entry);
-  if (cudaGetLastError() != cudaSuccess) {
-    p->fixed_mem = nullptr;
-    return fail(LOSA_ERR_CUDA);
-  }
-  cudaFreeAsync(scratch, stream);
+  if (cudaGetLastError() != cudaSuccess) return fail(LOSA_ERR_CUDA);
+  cudaFreeAsync(job.scratch, stream);
+  job = SelectJob{};
   *out = p;
   return LOSA_OK;
+}
+
+int build_pattern(const float* mass, int B, int H, int n, int block, double tau,
+                  losa_pattern** out, cudaStream_t stream) {
+  SelectJob job;
+  const int st = select_begin(B, H, n, block, tau, stream, job);
+  if (st != LOSA_OK) return st;
+  return select_end(mass, /*run_cut=*/true, job, out);
 }
 
 int import_pattern(const int32_t* row_ptr, const int32_t* col_idx, const int64_t* retained_fx,

@@ -17,6 +17,8 @@
  *                     Mask Generation; legiblepapers.com LoSA page, "Summary
  *                     & Methodology Analysis": default tau = 0.99), frozen
  *                     into a CSR pattern the library owns.
+ *   losa_dense_mass_select  the first two phases in one call, the per-row
+ *                     cut fused into the construction kernel.
  *   losa_sparse_attn  every later step: attention of fresh Q/K/V over the
  *                     frozen retained key blocks only (Phase 3 - Repeated
  *                     Sparse Inference; legiblepapers.com: Q, K, V are
@@ -34,7 +36,8 @@
  *   - Attention is bidirectional: softmax(scale * q k^T) over the valid keys.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *     stream-ordered and return without a host synchronisation, except
- *     losa_select (one synchronisation, to size the CSR),
+ *     losa_select and losa_dense_mass_select (one synchronisation, to size
+ *     the CSR),
  *     losa_pattern_export / losa_pattern_import (they finish their copies
  *     before returning) and losa_check_status.
  *   - Every call returns LOSA_OK (0) or a negative losa_status; it checks
@@ -152,6 +155,34 @@ int losa_dense_mass(const void* q, const void* k, const void* v, int in_dtype,
  */
 int losa_select(const float* mass, int B, int H, int n_blocks, int block, double tau,
                 losa_pattern** out, void* stream);
+
+/*
+ * losa_dense_mass_select - losa_dense_mass and losa_select in one call, with
+ * the selection's per-row cut run inside the construction kernel: a CTA of
+ * that kernel computes every key block of its query blocks' mass rows, so
+ * once its mass pass is over it sorts and cuts those rows itself (Phase 1
+ * and Phase 2 of the ubos.tech LoSA post, "How It Works in Practice"; the
+ * LoSA abstract's "smallest key/value block set" per head and query block).
+ * The tile lists and the tile order are then built as losa_select builds
+ * them.
+ *
+ *   Arguments as for losa_dense_mass (q, k, v, o, lse, mass and their
+ *   dtypes, shapes, alignment) plus tau and out as for losa_select.
+ *   o, lse and mass are written exactly as losa_dense_mass writes them, and
+ *   the pattern is bit-identical to losa_select(mass, ..., tau) on that
+ *   mass map (the same integer cut, run by one warpgroup per row instead
+ *   of one CTA or warp per row).
+ *   Synchronises the stream once (to size the CSR), like losa_select, and
+ *   allocates from the library's pool on `stream`.
+ *   Returns LOSA_ERR_ARG (as for losa_dense_mass, a null out, or tau outside
+ *   (0, 1]), LOSA_ERR_NOMEM, LOSA_ERR_CUDA, LOSA_ERR_TIMEOUT (the
+ *   construction kernel gave up a bounded wait; the status word is cleared
+ *   and no pattern is returned), LOSA_ERR_UNSUPPORTED.
+ */
+int losa_dense_mass_select(const void* q, const void* k, const void* v, int in_dtype,
+                           int B, int H, int L, int L_pad, int d, int block, float scale,
+                           double tau, void* o, int out_dtype, float* lse, float* mass,
+                           losa_pattern** out, void* stream);
 
 /* Fills *view from a pattern. Returns LOSA_ERR_ARG on NULL. */
 int losa_pattern_info(const losa_pattern* p, losa_pattern_view* view);

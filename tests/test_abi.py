@@ -79,6 +79,34 @@ def test_dense_mass_rejects_bad_arguments(losa, bad):
     assert _dense(losa.lib(), **bad) == -1
 
 
+def _dense_select(lib, tau=0.99, out=True, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, in_dt=0, B=1, H=2, L=250, L_pad=256, d=64, block=32,
+             scale=0.125, o=FAKE, out_dt=1, lse=FAKE, mass=FAKE, stream=None)
+    a.update(kw)
+    h = ctypes.c_void_p(123)
+    st = lib.losa_dense_mass_select(a["q"], a["k"], a["v"], a["in_dt"], a["B"], a["H"], a["L"],
+                                    a["L_pad"], a["d"], a["block"], a["scale"], tau, a["o"],
+                                    a["out_dt"], a["lse"], a["mass"],
+                                    ctypes.byref(h) if out else None, a["stream"])
+    return st, h.value
+
+
+@pytest.mark.parametrize("bad", [
+    dict(q=None), dict(mass=None), dict(lse=None), dict(o=None), dict(in_dt=7), dict(B=0),
+    dict(L=300), dict(L=200), dict(d=96), dict(block=16), dict(scale=0.0),
+    dict(L=70000, L_pad=70016, block=32), dict(B=300, H=300), dict(v=ctypes.c_void_p(0x10004)),
+    dict(tau=0.0), dict(tau=1.5), dict(tau=float("nan")), dict(out=False),
+])
+def test_dense_mass_select_rejects_bad_arguments(losa, bad):
+    """The fused call checks what losa_dense_mass and losa_select check
+    (shapes, dtypes, alignment, tau in (0, 1], a place for the pattern) on
+    the host, and leaves the pattern slot NULL when it refuses."""
+    st, h = _dense_select(losa.lib(), **bad)
+    assert st == -1
+    if bad != dict(out=False):
+        assert h is None
+
+
 @pytest.mark.parametrize("tau", [0.0, -0.5, 1.0000001, 2.0, float("nan")])
 def test_select_rejects_tau_outside_unit_interval(losa, tau):
     out = ctypes.c_void_p(123)
