@@ -112,6 +112,25 @@ template <int D> constexpr int poly_pairs_mass() { return 7; }
 constexpr int kCutSmemStride = 32768;
 static_assert(sizeof(cut::BucketSmem) <= kCutSmemStride, "cut workspace");
 
+// The fused cut of one warpgroup's mass rows: rows I0 .. I0 + nq - 1 of
+// head bh (those below n_blocks), tid the thread's index in the warpgroup
+// of tile t. Kept out of line, so that the kernel's main loops are compiled
+// as in the instances without it.
+__device__ __noinline__ void fused_cut_rows(const float* mass, int n, unsigned long long tau_fx,
+                                            unsigned long long* cut_key, int* count,
+                                            long long* retained_fx, long long* total_fx,
+                                            int* status, cut::BucketSmem* sm, int t, int tid,
+                                            int bh, int I0, int nq) {
+  const WarpgroupSync wg_sync{2 + t};
+  for (int q = 0; q < nq; ++q) {
+    const int I = I0 + q;
+    if (I >= n) break;
+    const int64_t mr = int64_t(bh) * n + I;
+    cut::bucket_cut_row<128>(mass + mr * n, n, tau_fx, *sm, tid, wg_sync, mr, cut_key, count,
+                             retained_fx, total_fx, status);
+  }
+}
+
 constexpr int kAttnThreads = 384;
 constexpr int kAttnLaunchRegs = 168;   // checked against ptxas at build time
 constexpr int kSoftmaxRegs = 216;
@@ -891,18 +910,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
         __threadfence_block();
         const bool quit = named_bar_or(1, 256, !ok || *abort_flag != 0);
-        if (!quit) {
-          auto& sm = *reinterpret_cast<cut::BucketSmem*>(smem + t * kCutSmemStride);
-          const WarpgroupSync wg_sync{2 + t};
-          for (int q = 0; q < BM / BLK; ++q) {
-            const int I = qt[t] * (BM / BLK) + q;
-            if (I >= p.n_blocks) break;
-            const int64_t mr = int64_t(bh[t]) * p.n_blocks + I;
-            cut::bucket_cut_row<128>(p.mass + mr * p.n_blocks, p.n_blocks, p.tau_fx, sm, r,
-                                     wg_sync, mr, p.cut_key, p.cut_count, p.retained_fx,
-                                     p.total_fx, p.status);
-          }
-        }
+        if (!quit)
+          fused_cut_rows(p.mass, p.n_blocks, p.tau_fx, p.cut_key, p.cut_count, p.retained_fx,
+                         p.total_fx, p.status,
+                         reinterpret_cast<cut::BucketSmem*>(smem + t * kCutSmemStride), t, r,
+                         bh[t], qt[t] * (BM / BLK), BM / BLK);
       }
     }
   }
