@@ -43,6 +43,7 @@ METRIC = ("block-sparse attn ms & TFLOP/s (retained blocks), % BF16 TC peak; "
           "mass+select ms")
 DEFAULT_WORKLOAD = "hunyuanvideo"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tensor-core rates of B200
 # Kernels the library launches per call: dense_mass 1 (bf16 inputs), select 8, sparse 1.
 LAUNCHES_DENSE, LAUNCHES_SELECT, LAUNCHES_SPARSE = 1, 8, 1
 
@@ -63,6 +64,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused construction + selection comparison")
+    ap.add_argument("--fp32-inputs", action="store_true",
+                    help="hand the library fp32 Q/K/V (the kind::tf32 kernels; each call "
+                         "rounds its inputs to tf32 first); roofline against the tf32 peak")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small profiling cases)")
     ap.add_argument("--ncu-case", action="store_true",
@@ -240,7 +244,8 @@ def oracle_sample(wl, tau, n_sparse, budget_s, seed=4321, max_sets=4):
 def distinct_sets(wl, n_sparse):
     """How many distinct drifted input sets stay resident (at most ~16 GB);
     longer runs cycle through them."""
-    set_bytes = 3 * wl.batch * wl.heads * wl.seq_pad * wl.head_dim * 2
+    esz = 4 if wl.in_dtype == "fp32" else 2
+    set_bytes = 3 * wl.batch * wl.heads * wl.seq_pad * wl.head_dim * esz
     return max(1, min(n_sparse, int(16e9 // set_bytes)))
 
 
@@ -251,7 +256,7 @@ def bench_config(wl, tau, n_sparse, world):
             "seq_len": wl.seq_len, "seq_pad": Lp, "block": wl.block, "tau": tau,
             "sparse_steps": n_sparse, "distinct_step_inputs": distinct_sets(wl, n_sparse),
             "l2": "inputs larger than L2 (3 x "
-                  f"{B * H * Lp * d * 2 / 1e6:.0f} MB per call)",
+                  f"{B * H * Lp * d * (4 if wl.in_dtype == 'fp32' else 2) / 1e6:.0f} MB per call)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -539,6 +544,8 @@ def main():
     wl = W.WORKLOADS[args.workload]
     if args.heads is not None:
         wl = dataclasses.replace(wl, heads=args.heads)
+    if args.fp32_inputs:
+        wl = dataclasses.replace(wl, in_dtype="fp32")
     if args.tau_sweep or args.stability or args.sched_analysis:
         dev = torch.device("cuda", local)
         if args.tau_sweep:
@@ -643,6 +650,11 @@ def main():
     # bf16 figure; the fraction of the burst figure is reported beside it.
     peak = peaks["bf16_tflops_sustained"]
     burst = peaks["bf16_tflops"]
+    peak_dtype = "bf16"
+    if wl.in_dtype == "fp32":
+        # kind::tf32 kernels: the measured bf16 peaks times the nominal dense
+        # tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s)
+        peak, burst, peak_dtype = peak * TF32_PER_BF16, burst * TF32_PER_BF16, "tf32"
     value = world * f_step / (step_ms * 1e-3) / 1e12
     sparse_tf = f_sparse / (sparse_ms * 1e-3) / 1e12
     dense_tf = f_dense / (dense_ms * 1e-3) / 1e12
@@ -652,7 +664,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": step_ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "tf32" if wl.in_dtype == "fp32" else "bf16",
         "data": "synthetic",
         "config": bench_config(wl, tau, n_sparse, world),
         "sparse_attn": {"ms": sparse_ms, "tflops": sparse_tf, "frac_of_peak": sparse_tf / peak,
@@ -669,10 +682,14 @@ def main():
         "sparse_vs_dense_speedup": (dense_ms * 4.0 / 6.0) / sparse_ms,
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": sparse_tf,
                      "peak": peak, "unit": "TFLOP/s", "frac": sparse_tf / peak,
-                     "traffic": measured_traffic(wl.name) if args.heads is None else None,
+                     "traffic": measured_traffic(wl.name)
+                     if args.heads is None and wl.in_dtype != "fp32" else None,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a "
-                                    f"long step); frac of the burst figure {burst:.1f}: "
-                                    f"{sparse_tf / burst:.3f}"},
+                                    f"long step)"
+                                    + (f" x {TF32_PER_BF16:.3f} (nominal dense tf32 / bf16)"
+                                       if peak_dtype == "tf32" else "")
+                                    + f"; frac of the burst figure {burst:.1f}: "
+                                      f"{sparse_tf / burst:.3f}"},
         "gpu_launches": args.steps * (LAUNCHES_DENSE + LAUNCHES_SELECT + n_sparse * LAUNCHES_SPARSE),
         "clocks": clock_info,
     }
