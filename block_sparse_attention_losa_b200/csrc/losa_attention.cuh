@@ -907,6 +907,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // free for the cut's workspace, and the barrier makes the mass rows
         // these warps wrote visible to them. A warp that gave up a wait, or
         // an abort anywhere in the CTA, skips the cut in both warpgroups.
+        // Named barriers: 1 joins the two softmax warpgroups (256 threads),
+        // 2 + t the warpgroup of tile t inside the cut; barrier 0 stays the
+        // CTA-wide one at the end of the kernel.
         __syncwarp();
         __threadfence_block();
         const bool quit = named_bar_or(1, 256, !ok || *abort_flag != 0);
